@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 W4A4 matmul on B200 (one JSON line on rank 0).
+
+Workload: the FFN down projection, Y[4096,5376] = A[4096,14336] . W[5376,14336]^T
+in NVFP4 (two-level quantisation of N(0,1) activations and N(0,0.02) weights,
+seeded).  A step is one call of gemm_nvfp4_w4a4 on device-resident inputs.
+L2 is flushed (a 256 MiB write) between timed steps, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun, one process per GPU) every rank runs its own
+batch of the same shape (data parallel, weak scaling, no collective on the
+data path); the per-step device time is the max over ranks.
+
+`--impl reference` times the FP64 CPU oracle instead (rank 0 only; each step is
+a bounded sample of rows of the same workload), for the driver's ratio.
+`--workload` picks another path for profiling runs only; its line is not the
+headline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 W4A4 GEMM TFLOPS at M4096 N5376 K14336; % of B200 dense FP4 peak"
+FP4_PER_BF16 = 9.0 / 2.25          # nominal dense FP4 : BF16 tensor ratio
+FALLBACK_BF16_TFLOPS = 1590.0      # used only if MEASURED_PEAKS.json is absent
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=["ffn_down", "tiny"], default="ffn_down")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+
+
+def make_workload(name):
+    from block_scaled_precision_nvfp4_b200 import workloads as wl
+    if name == "tiny":
+        return wl.tiny_w4a4(0)
+    return wl.ffn_down_w4a4()
+
+
+# --- clock sampling during the timed region (NVML reads only) -------------------------
+
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
+        0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown",
+        0x200: "display_clock_setting"}
+
+    def __init__(self, torch_dev):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+            self.h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    self.h = h
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(torch_dev)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - no NVML
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": len(self.samples)}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and bit != 0x1]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# --- the reference arm: the FP64 oracle on the host cores ------------------------------
+
+def oracle_rows_for(seconds, wl_, rate_probe_rows=4):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.gemm_w4a4(wl_.A.codes[:rate_probe_rows], wl_.A.scales[:rate_probe_rows], wl_.A.g,
+                     wl_.W.codes, wl_.W.scales, wl_.W.g, rate_probe_rows, wl_.N, wl_.K)
+    rate = rate_probe_rows / max(time.perf_counter() - t0, 1e-6)  # rows per second
+    return int(max(1, min(wl_.M, round(rate * seconds))))
+
+
+def time_oracle(wl_, rows):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.gemm_w4a4(wl_.A.codes[:rows], wl_.A.scales[:rows], wl_.A.g, wl_.W.codes,
+                     wl_.W.scales, wl_.W.g, rows, wl_.N, wl_.K)
+    dt = time.perf_counter() - t0
+    return 2.0 * rows * wl_.N * wl_.K / dt / 1e12, dt
+
+
+def cpu_baseline(wl_, seconds=12.0):
+    import oracle
+    rows = oracle_rows_for(seconds, wl_)
+    tflops, dt = time_oracle(wl_, rows)
+    return {"value": tflops, "unit": "TFLOP/s", "cores": oracle.default_threads(),
+            "kind": "oracle",
+            "sample": f"first {rows} of {wl_.M} rows of Y ({rows}x{wl_.N}x{wl_.K}), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    wl_ = make_workload(args.workload)
+    rows = oracle_rows_for(1.0, wl_)
+    for _ in range(args.warmup):
+        time_oracle(wl_, rows)
+    times = []
+    for _ in range(args.steps):
+        _, dt = time_oracle(wl_, rows)
+        times.append(dt)
+    t = sum(times) / len(times)
+    value = 2.0 * rows * wl_.N * wl_.K / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl_.name, "M": wl_.M, "N": wl_.N, "K": wl_.K,
+                   "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "kind": "oracle",
+                         "cores": oracle.default_threads(),
+                         "sample": f"first {rows} of {wl_.M} rows of Y per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --- our arm ---------------------------------------------------------------------------
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_scaled_precision_nvfp4_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for ln in f:
+                if ":" in ln:
+                    k, v = ln.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("source_hash") == kernel_source_hash():
+            return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import block_scaled_precision_nvfp4_b200 as nv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+    nv.load_library(build_if_missing=False)
+
+    wl_ = make_workload(args.workload)
+    M, N, K = wl_.M, wl_.N, wl_.K
+    flops = 2.0 * M * N * K
+
+    def dev_(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+
+    A, sA, W, sW = dev_(wl_.A.codes), dev_(wl_.A.scales), dev_(wl_.W.codes), dev_(wl_.W.scales)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        nv.gemm_nvfp4_w4a4(A, sA, wl_.A.g, W, sW, wl_.W.g, out=Y, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    nv.nvfp4_check_device_error(stream)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    nv.nvfp4_check_device_error(stream)
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
+    t_ms = sum(per_step) / len(per_step)
+    if world > 1:
+        tt = torch.tensor([t_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ms = float(tt.item())
+    value = world * flops / (t_ms * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device -> call -> host result
+    e2e = None
+    if not args.no_e2e:
+        hA, hsA, hW, hsW = (torch.from_numpy(np.ascontiguousarray(x)).pin_memory() for x in
+                            (wl_.A.codes, wl_.A.scales, wl_.W.codes, wl_.W.scales))
+        hY = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        e_steps = max(1, min(args.steps, 20))
+
+        def e2e_step():
+            A.copy_(hA, non_blocking=True); sA.copy_(hsA, non_blocking=True)
+            W.copy_(hW, non_blocking=True); sW.copy_(hsW, non_blocking=True)
+            step()
+            hY.copy_(Y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        te = e0.elapsed_time(e1) / e_steps
+        if world > 1:
+            tt = torch.tensor([te], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            te = float(tt.item())
+        h2d = sum(x.numel() * x.element_size() for x in (hA, hsA, hW, hsW))
+        e2e = {"value": world * flops / (te * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hY.numel() * 2,
+               "ms_per_step": te}
+
+    bf16_peak, _, peak_src = peaks()
+    fp4_peak = bf16_peak * FP4_PER_BF16
+    achieved = flops / (t_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4(e2m1 x e2m1, e4m3 group scales) -> f32 accumulate -> bf16",
+        "data": "synthetic",
+        "config": {"workload": wl_.name, "M": M, "N": N, "K": K, "global_batch": world * M,
+                   "parallelism": f"dp{world}", "l2": "flushed between timed steps (256 MiB write)",
+                   "inputs": wl_.notes},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+                     "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                     "peak_note": f"{peak_src} bf16 {bf16_peak:.1f} TFLOP/s x nominal fp4/bf16 4",
+                     "traffic": profiled_traffic(wl_.name),
+                     "kernel": "w4a4_kernel<256,4>",
+                     "per_launch_ms": {"median": statistics.median(per_step),
+                                       "min": min(per_step)}},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl_)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

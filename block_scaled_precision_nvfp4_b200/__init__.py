@@ -1,0 +1,262 @@
+"""B200 (sm_100a) block-scaled NVFP4 matmul: Python binding of the C ABI in include/nvfp4.h.
+
+The names mirror the C entry points.  This module only marshals arguments:
+torch tensors (CUDA memory, allocated by PyTorch) become raw pointers and the
+current torch stream becomes the ``stream`` argument; every step of the
+computation runs in the library's own kernels.  There is no CPU fallback: on a
+machine whose library cannot load, or whose device has no path, each call
+raises.
+
+Formats (metrale_circuit ``hardware::exec`` module doc, bullets 1-2):
+packed E2M1 codes ``uint8[rows, K/2]`` (even k in the low nibble), E4M3 group
+scales ``uint8[rows, K/16]`` (one per 16 consecutive k), FP32 per-tensor scales,
+BF16 output ``[M, N]`` = alpha * (A.sA)(W.sW)^T.
+"""
+from __future__ import annotations
+
+import ctypes
+import enum
+import os
+import threading
+
+from . import _build
+
+__all__ = [
+    "Fmt", "Kind", "Exec", "Status", "NvFp4Error", "load_library", "library_path",
+    "nvfp4_kind_of", "nvfp4_exec_of", "nvfp4_exec_of_arch", "nvfp4_pair_name",
+    "nvfp4_exec_name", "nvfp4_set_fp4_kernel_disabled", "nvfp4_version",
+    "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_w4a16",
+    "nvfp4_w4a16_workspace_size", "gemm_nvfp4_w4a4_grouped", "C_FUNCTIONS",
+]
+
+
+class Fmt(enum.IntEnum):
+    BF16 = 0
+    FP8_E4M3 = 1
+    NVFP4 = 2
+
+
+class Kind(enum.IntEnum):
+    BF16_MMA = 0
+    FP8_MMA = 1
+    FP4_BLOCK_SCALED = 2
+    INVALID = -1
+
+
+class Exec(enum.IntEnum):
+    FP4_MMA = 0
+    FP8_EXACT = 1
+    BF16_WIDEN = 2
+    NO_FP4_KERNEL = 3
+    NO_PATH = 4
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    INVALID_ARG = 1
+    MISALIGNED = 2
+    NOPATH = 3
+    NO_FP4_KERNEL = 4
+    CUDA = 5
+    DEVICE_TIMEOUT = 6
+
+
+class NvFp4Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = Status(status)
+        super().__init__(f"{self.status.name}: {message}")
+
+
+# C signatures: name -> (restype, argtypes)
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_S = ctypes.c_char_p
+C_FUNCTIONS = {
+    "nvfp4_version": (_S, []),
+    "nvfp4_last_error": (_S, []),
+    "nvfp4_kind_of": (_I, [_I]),
+    "nvfp4_exec_of_arch": (_I, [_I, _I, _I, _I]),
+    "nvfp4_exec_of": (_I, [_I, _I, _I]),
+    "nvfp4_set_fp4_kernel_disabled": (None, [_I]),
+    "nvfp4_pair_name": (_S, [_I, _I]),
+    "nvfp4_exec_name": (_S, [_I]),
+    "nvfp4_check_device_error": (_I, [_P]),
+    "gemm_nvfp4_w4a4": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
+    "gemm_nvfp4_via_fp8": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
+    "gemm_w4a16": (_I, [_P, _P, _P, _F, _P, _I, _I, _I, _P, _Z, _P]),
+    "nvfp4_w4a16_workspace_size": (_Z, [_I, _I, _I]),
+    "gemm_nvfp4_w4a4_grouped": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libnvfp4_b200.so (building it with nvcc if absent).  Raises if it cannot load."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_build.LIB):
+                if not build_if_missing:
+                    raise OSError(f"{_build.LIB} is missing; run block_scaled_precision_nvfp4_b200."
+                                  "_build.build()")
+                _build.build()
+            lib = ctypes.CDLL(_build.LIB)
+            for name, (res, args) in C_FUNCTIONS.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _err(status: int):
+    if status != 0:
+        msg = load_library().nvfp4_last_error().decode(errors="replace")
+        raise NvFp4Error(status, msg)
+
+
+# --- planning -------------------------------------------------------------------
+
+def nvfp4_version() -> str:
+    return load_library().nvfp4_version().decode()
+
+
+def nvfp4_kind_of(activation: Fmt) -> Kind:
+    return Kind(load_library().nvfp4_kind_of(int(activation)))
+
+
+def nvfp4_exec_of_arch(sm_arch: int, weight: Fmt, activation: Fmt,
+                       fp4_kernel_disabled: bool = False) -> Exec:
+    return Exec(load_library().nvfp4_exec_of_arch(int(sm_arch), int(weight), int(activation),
+                                                  int(bool(fp4_kernel_disabled))))
+
+
+def nvfp4_exec_of(device: int, weight: Fmt, activation: Fmt) -> Exec:
+    return Exec(load_library().nvfp4_exec_of(int(device), int(weight), int(activation)))
+
+
+def nvfp4_set_fp4_kernel_disabled(disabled: bool) -> None:
+    load_library().nvfp4_set_fp4_kernel_disabled(int(bool(disabled)))
+
+
+def nvfp4_pair_name(weight: Fmt, activation: Fmt) -> str:
+    return load_library().nvfp4_pair_name(int(weight), int(activation)).decode()
+
+
+def nvfp4_exec_name(e: Exec) -> str:
+    return load_library().nvfp4_exec_name(int(e)).decode()
+
+
+# --- tensor marshalling -----------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(stream=None) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _dev_tensor(t, dtype, shape, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device (there is no CPU path)")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def nvfp4_check_device_error(stream=None) -> None:
+    _err(load_library().nvfp4_check_device_error(_stream_ptr(stream)))
+
+
+# --- matmuls ----------------------------------------------------------------------
+
+def _w4a4_common(fn_name, A, sA, gA, W, sW, gW, out, stream):
+    torch = _torch()
+    M, half_k = A.shape
+    N = W.shape[0]
+    K = 2 * half_k
+    pa = _dev_tensor(A, torch.uint8, (M, K // 2), "A")
+    psa = _dev_tensor(sA, torch.uint8, (M, K // 16), "sA")
+    pw = _dev_tensor(W, torch.uint8, (N, K // 2), "W")
+    psw = _dev_tensor(sW, torch.uint8, (N, K // 16), "sW")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
+    _err(getattr(load_library(), fn_name)(pa, psa, float(gA), pw, psw, float(gW), py, M, N, K,
+                                          _stream_ptr(stream)))
+    return out
+
+
+def gemm_nvfp4_w4a4(A, sA, gA, W, sW, gW, out=None, stream=None):
+    """Y[M,N] (bf16) = gA*gW * (A.sA)(W.sW)^T on the block-scaled FP4 MMA."""
+    return _w4a4_common("gemm_nvfp4_w4a4", A, sA, gA, W, sW, gW, out, stream)
+
+
+def gemm_nvfp4_via_fp8(A, sA, gA, W, sW, gW, out=None, stream=None):
+    """The same product through the exact E2M1->E4M3 conversion on the FP8 MMA."""
+    return _w4a4_common("gemm_nvfp4_via_fp8", A, sA, gA, W, sW, gW, out, stream)
+
+
+def nvfp4_w4a16_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load_library().nvfp4_w4a16_workspace_size(int(M), int(N), int(K)))
+
+
+def gemm_w4a16(A, W, sW, gW, out=None, workspace=None, stream=None):
+    """Y[M,N] (bf16) = gW * A_bf16 . (W.sW)^T, weights widened to BF16 in registers."""
+    torch = _torch()
+    M, K = A.shape
+    N = W.shape[0]
+    pa = _dev_tensor(A, torch.bfloat16, (M, K), "A")
+    pw = _dev_tensor(W, torch.uint8, (N, K // 2), "W")
+    psw = _dev_tensor(sW, torch.uint8, (N, K // 16), "sW")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
+    need = nvfp4_w4a16_workspace_size(M, N, K)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=A.device)
+    pws = 0 if workspace is None else workspace.data_ptr()
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _err(load_library().gemm_w4a16(pa, pw, psw, float(gW), py, M, N, K, pws, wsb,
+                                   _stream_ptr(stream)))
+    return out
+
+
+def gemm_nvfp4_w4a4_grouped(A, sA, gA, W, sW, gW, offsets, out=None, stream=None):
+    """Grouped W4A4: W [E,N,K/2], sW [E,N,K/16], gW (E floats), offsets (E+1 ints, host)."""
+    torch = _torch()
+    M, half_k = A.shape
+    K = 2 * half_k
+    E, N = W.shape[0], W.shape[1]
+    pa = _dev_tensor(A, torch.uint8, (M, K // 2), "A")
+    psa = _dev_tensor(sA, torch.uint8, (M, K // 16), "sA")
+    pw = _dev_tensor(W, torch.uint8, (E, N, K // 2), "W")
+    psw = _dev_tensor(sW, torch.uint8, (E, N, K // 16), "sW")
+    off = (ctypes.c_int32 * (E + 1))(*[int(x) for x in offsets])
+    gws = (ctypes.c_float * E)(*[float(x) for x in gW])
+    if len(offsets) != E + 1 or int(offsets[-1]) != M:
+        raise ValueError("offsets must hold E+1 row offsets ending at A.shape[0]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
+    _err(load_library().gemm_nvfp4_w4a4_grouped(pa, psa, float(gA), pw, psw,
+                                                ctypes.cast(gws, ctypes.c_void_p),
+                                                ctypes.cast(off, ctypes.c_void_p), E, py, N, K,
+                                                _stream_ptr(stream)))
+    return out

@@ -1,0 +1,310 @@
+// nvfp4_api.cu -- the C ABI of include/nvfp4.h: argument checks, the exec_of
+// planner (metrale_circuit `hardware::exec`: Exec, exec_of, fp4_fallback,
+// kind_of, pair_name), tensor-map encoding and kernel launches.
+//
+// This is the only translation unit of the library; every kernel header is
+// included here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/nvfp4.h"
+#include "ptx.cuh"
+#include "w4a4_kernel.cuh"
+
+namespace {
+
+thread_local char t_last_error[512] = "";
+std::atomic<int> g_fp4_kernel_disabled{0};
+
+nvfp4_status fail(nvfp4_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+nvfp4_status ok() {
+    t_last_error[0] = '\0';
+    return NVFP4_OK;
+}
+
+nvfp4_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(NVFP4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- device info
+struct DevInfo {
+    bool valid = false;
+    int sm_arch = 0;     // 10*major + minor
+    int num_sms = 0;
+    size_t smem_optin = 0;
+};
+
+std::mutex g_dev_mu;
+DevInfo g_dev[64];
+
+bool device_info(int dev, DevInfo& out) {
+    if (dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!g_dev[dev].valid) {
+        int major = 0, minor = 0, sms = 0, smem = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        g_dev[dev].sm_arch = major * 10 + minor;
+        g_dev[dev].num_sms = sms;
+        g_dev[dev].smem_optin = (size_t)smem;
+        g_dev[dev].valid = true;
+    }
+    out = g_dev[dev];
+    return true;
+}
+
+bool current_device(int& dev, DevInfo& info) {
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return device_info(dev, info);
+}
+
+// ---------------------------------------------------------------- planner
+// Device classes that carry the block-scaled FP4 MMA instruction.
+bool class_has_fp4_mma(int arch) {
+    return arch == 100 || arch == 101 || arch == 103 || arch == 110 || arch == 120 || arch == 121;
+}
+// ... and the FP8 MMA.
+bool class_has_fp8_mma(int arch) { return arch >= 89; }
+// Classes this library compiles its kernels for (sm_100a code runs on CC 10.0 only).
+bool class_compiles_fp4_kernel(int arch) { return arch == 100; }
+bool class_compiles_fp8_exact_kernel(int arch) { return arch == 100; }
+bool class_compiles_bf16_widen_kernel(int arch) { return arch == 100; }
+
+// fp4_fallback: an NVFP4 activation on a class without an FP4 block-scale
+// kernel.  NoFp4Kernel where the class has the FP4 MMA and only the kernel is
+// missing; else the exact FP8 path where the class has the FP8 MMA (and this
+// library's exact-path kernel); else no path.
+nvfp4_exec fp4_fallback(int arch) {
+    if (class_has_fp4_mma(arch)) return NVFP4_EXEC_NO_FP4_KERNEL;
+    if (class_has_fp8_mma(arch) && class_compiles_fp8_exact_kernel(arch)) return NVFP4_EXEC_FP8_EXACT;
+    return NVFP4_EXEC_NO_PATH;
+}
+
+bool valid_fmt(nvfp4_fmt f) {
+    return f == NVFP4_FMT_BF16 || f == NVFP4_FMT_FP8_E4M3 || f == NVFP4_FMT_NVFP4;
+}
+
+// Launch-time check shared by the W4A4 entry points.
+nvfp4_status check_fp4_path(int& dev, DevInfo& info) {
+    if (!current_device(dev, info)) return fail(NVFP4_ERR_CUDA, "cannot query the current CUDA device");
+    nvfp4_exec e = nvfp4_exec_of_arch(info.sm_arch, NVFP4_FMT_NVFP4, NVFP4_FMT_NVFP4,
+                                      g_fp4_kernel_disabled.load());
+    if (e == NVFP4_EXEC_FP4_MMA) return NVFP4_OK;
+    if (e == NVFP4_EXEC_NO_FP4_KERNEL)
+        return fail(NVFP4_ERR_NO_FP4_KERNEL,
+                    "sm_%d has the FP4 MMA but no FP4 block-scale kernel is compiled for it",
+                    info.sm_arch);
+    return fail(NVFP4_ERR_NOPATH, "W4A4 has no FP4 MMA path on sm_%d (plan: %s)", info.sm_arch,
+                nvfp4_exec_name(e));
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        cudaGetLastError();
+    });
+    return g_encode != nullptr;
+}
+
+// 2D uint8 map over a row-major [rows][row_bytes] buffer, box [box_rows][box_bytes],
+// 128-byte swizzle (box_bytes must be 128), zero fill out of bounds.
+nvfp4_status make_map_u8(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
+                         uint32_t box_bytes, uint32_t box_rows) {
+    if (!get_encoder()) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {row_bytes, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_bytes, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return NVFP4_OK;
+}
+
+// ---------------------------------------------------------------- argument checks
+nvfp4_status check_w4a4_args(const void* A, const void* sA, const void* W, const void* sW,
+                             const void* Y, int M, int N, int K) {
+    if (M < 0 || N < 0) return fail(NVFP4_ERR_INVALID_ARG, "M and N must be >= 0 (got %d, %d)", M, N);
+    if (K < 32 || K % 32 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "K must be a positive multiple of 32 (got %d)", K);
+    if (M == 0 || N == 0) return NVFP4_OK;
+    if (!A || !sA || !W || !sW || !Y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(A) || !aligned16(sA) || !aligned16(W) || !aligned16(sW) || !aligned16(Y))
+        return fail(NVFP4_ERR_MISALIGNED, "every buffer must be 16-byte aligned");
+    return NVFP4_OK;
+}
+
+template <typename Kern>
+nvfp4_status set_smem(Kern k, size_t bytes, const DevInfo& info, const char* name) {
+    if (bytes > info.smem_optin)
+        return fail(NVFP4_ERR_CUDA, "%s needs %zu B of shared memory, device allows %zu", name,
+                    bytes, info.smem_optin);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return cuda_fail(e, name);
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+const char* nvfp4_version(void) { return "nvfp4-b200 0.1 (sm_100a)"; }
+
+const char* nvfp4_last_error(void) { return t_last_error; }
+
+nvfp4_kind nvfp4_kind_of(nvfp4_fmt activation) {
+    switch (activation) {
+    case NVFP4_FMT_BF16: return NVFP4_KIND_BF16_MMA;
+    case NVFP4_FMT_FP8_E4M3: return NVFP4_KIND_FP8_MMA;
+    case NVFP4_FMT_NVFP4: return NVFP4_KIND_FP4_BLOCK_SCALED;
+    }
+    return NVFP4_KIND_INVALID;
+}
+
+const char* nvfp4_pair_name(nvfp4_fmt weight, nvfp4_fmt activation) {
+    static const char* names[3][3] = {
+        {"W16A16", "W16A8", "W16A4"}, {"W8A16", "W8A8", "W8A4"}, {"W4A16", "W4A8", "W4A4"}};
+    if (!valid_fmt(weight) || !valid_fmt(activation)) return "?";
+    return names[weight][activation];
+}
+
+const char* nvfp4_exec_name(nvfp4_exec e) {
+    switch (e) {
+    case NVFP4_EXEC_FP4_MMA: return "FP4_MMA";
+    case NVFP4_EXEC_FP8_EXACT: return "FP8_EXACT";
+    case NVFP4_EXEC_BF16_WIDEN: return "BF16_WIDEN";
+    case NVFP4_EXEC_NO_FP4_KERNEL: return "NO_FP4_KERNEL";
+    case NVFP4_EXEC_NO_PATH: return "NO_PATH";
+    }
+    return "?";
+}
+
+nvfp4_exec nvfp4_exec_of_arch(int arch, nvfp4_fmt weight, nvfp4_fmt activation,
+                              int fp4_kernel_disabled) {
+    if (!valid_fmt(weight) || !valid_fmt(activation)) return NVFP4_EXEC_NO_PATH;
+    if (weight != NVFP4_FMT_NVFP4) return NVFP4_EXEC_NO_PATH;  // NVFP4-weight paths only
+    switch (nvfp4_kind_of(activation)) {
+    case NVFP4_KIND_FP4_BLOCK_SCALED:
+        if (class_has_fp4_mma(arch) && class_compiles_fp4_kernel(arch) && !fp4_kernel_disabled)
+            return NVFP4_EXEC_FP4_MMA;
+        return fp4_fallback(arch);
+    case NVFP4_KIND_BF16_MMA:
+        return class_compiles_bf16_widen_kernel(arch) ? NVFP4_EXEC_BF16_WIDEN : NVFP4_EXEC_NO_PATH;
+    case NVFP4_KIND_FP8_MMA:
+        // W4A8 has no single-instruction MMA; its exact E4M3 path is not carried yet.
+        return NVFP4_EXEC_NO_PATH;
+    default:
+        return NVFP4_EXEC_NO_PATH;
+    }
+}
+
+nvfp4_exec nvfp4_exec_of(int device, nvfp4_fmt weight, nvfp4_fmt activation) {
+    DevInfo info;
+    if (!device_info(device, info)) return NVFP4_EXEC_NO_PATH;
+    return nvfp4_exec_of_arch(info.sm_arch, weight, activation, g_fp4_kernel_disabled.load());
+}
+
+void nvfp4_set_fp4_kernel_disabled(int disabled) { g_fp4_kernel_disabled.store(disabled ? 1 : 0); }
+
+nvfp4_status nvfp4_check_device_error(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, nvfp4::g_device_error, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (v == 0) return ok();
+    e = cudaMemcpyToSymbol(nvfp4::g_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    return fail(NVFP4_ERR_DEVICE_TIMEOUT, "a kernel wait expired (role %d)", (v >> 8) & 0xFF);
+}
+
+// ------------------------------------------------------------------------- W4A4
+nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, float gA, const uint8_t* W,
+                             const uint8_t* sW, float gW, void* Y, int M, int N, int K,
+                             void* stream) {
+    nvfp4_status st = check_w4a4_args(A, sA, W, sW, Y, M, N, K);
+    if (st != NVFP4_OK) return st;
+    int dev;
+    DevInfo info;
+    if ((st = check_fp4_path(dev, info)) != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return ok();
+
+    constexpr int BN = 256, STAGES = 4;
+    using C = nvfp4::w4a4::Cfg<BN, STAGES>;
+    auto kern = nvfp4::w4a4::w4a4_kernel<BN, STAGES>;
+    CUtensorMap tmA, tmB;
+    if ((st = make_map_u8(&tmA, A, (uint64_t)K / 2, (uint64_t)M, nvfp4::w4a4::BKB,
+                          nvfp4::w4a4::BM)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_u8(&tmB, W, (uint64_t)K / 2, (uint64_t)N, nvfp4::w4a4::BKB, BN)) != NVFP4_OK)
+        return st;
+    if ((st = set_smem(kern, C::SMEM_BYTES, info, "w4a4_kernel")) != NVFP4_OK) return st;
+
+    const int tiles = ((M + nvfp4::w4a4::BM - 1) / nvfp4::w4a4::BM) * ((N + BN - 1) / BN);
+    const int grid = tiles < info.num_sms ? tiles : info.num_sms;
+    kern<<<grid, nvfp4::w4a4::NUM_THREADS, C::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
+        tmA, tmB, sA, sW, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launching w4a4_kernel");
+    return ok();
+}
+
+// ------------------------------------------------------------------------- not yet built
+nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, float, const uint8_t* W,
+                                const uint8_t* sW, float, void* Y, int M, int N, int K, void*) {
+    nvfp4_status st = check_w4a4_args(A, sA, W, sW, Y, M, N, K);
+    if (st != NVFP4_OK) return st;
+    return fail(NVFP4_ERR_NOPATH, "gemm_nvfp4_via_fp8 is not built yet");
+}
+
+nvfp4_status gemm_w4a16(const void*, const uint8_t*, const uint8_t*, float, void*, int, int, int,
+                        void*, size_t, void*) {
+    return fail(NVFP4_ERR_NOPATH, "gemm_w4a16 is not built yet");
+}
+
+size_t nvfp4_w4a16_workspace_size(int, int, int) { return 0; }
+
+nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t*, const uint8_t*, float, const uint8_t*,
+                                     const uint8_t*, const float*, const int32_t*, int, void*, int,
+                                     int, void*) {
+    return fail(NVFP4_ERR_NOPATH, "gemm_nvfp4_w4a4_grouped is not built yet");
+}
+
+}  // extern "C"

@@ -1,0 +1,192 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) block-scaled NVFP4 matmul library.
+ *
+ * The operation (metrale_circuit `hardware::exec` module doc, bullets 1-2; the
+ * NVFP4 formats it names):
+ *
+ *     Y[m,n] = BF16( alpha * sum_g sA[m,g]*sW[n,g] * sum_{k in g} a[m,k]*w[n,k] )
+ *
+ * where a, w are E2M1 (FP4) values, g runs over groups of 16 consecutive k,
+ * sA, sW are E4M3 group scales, alpha = gA*gW is the product of the two FP32
+ * per-tensor scales, accumulation is FP32 and the output is BF16 (round to
+ * nearest even).  The declared formats are never widened ("no silent upcast",
+ * module doc, Invariants): a pair with no native or exact path is reported as
+ * NVFP4_EXEC_NO_PATH and every matmul entry point refuses it.
+ *
+ * Layouts (all row-major, contiguous, no padding):
+ *   A      uint8 [M][K/2]   E2M1 codes, two per byte, even k in the low nibble
+ *   W      uint8 [N][K/2]   same; W is stored [N,K] so Y = A . W^T (TN)
+ *   sA     uint8 [M][K/16]  E4M3 group scales, finite and non-negative (0x00..0x7E)
+ *   sW     uint8 [N][K/16]  same
+ *   Y      bf16  [M][N]
+ * Every pointer is a DEVICE pointer, owned by the caller, and must be 16-byte
+ * aligned.  The library allocates no device memory in any call; kernels
+ * allocate and free their own tensor memory (TMEM) on chip.
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default
+ * stream).  NVFP4_OK means "enqueued".  Argument errors are detected on the
+ * host before anything is enqueued.  A kernel whose internal wait exceeds its
+ * time limit records a device error word and exits without hanging; it is
+ * read (and cleared) by nvfp4_check_device_error().
+ *
+ * Thread safety: every entry point may be called from several host threads;
+ * the only global state is a mutex-protected per-device capability cache and
+ * the per-thread last-error string.
+ */
+#ifndef NVFP4_B200_H
+#define NVFP4_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,     /* bad size, null pointer, bad enum, K % 32 != 0 ... */
+    NVFP4_ERR_MISALIGNED = 2,      /* a pointer is not 16-byte aligned */
+    NVFP4_ERR_NOPATH = 3,          /* the declared pair has no path on this device */
+    NVFP4_ERR_NO_FP4_KERNEL = 4,   /* device has the FP4 MMA but no kernel is compiled for it */
+    NVFP4_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed (see nvfp4_last_error) */
+    NVFP4_ERR_DEVICE_TIMEOUT = 6   /* a kernel's bounded wait expired (nvfp4_check_device_error) */
+} nvfp4_status;
+
+/* Declared operand formats (module doc, bullet 1: the activation format picks
+ * the MMA kind). */
+typedef enum {
+    NVFP4_FMT_BF16 = 0,
+    NVFP4_FMT_FP8_E4M3 = 1,
+    NVFP4_FMT_NVFP4 = 2
+} nvfp4_fmt;
+
+/* The MMA kind an activation format needs (`kind_of`). */
+typedef enum {
+    NVFP4_KIND_BF16_MMA = 0,       /* BF16 activations; weights widened in registers */
+    NVFP4_KIND_FP8_MMA = 1,
+    NVFP4_KIND_FP4_BLOCK_SCALED = 2,
+    NVFP4_KIND_INVALID = -1
+} nvfp4_kind;
+
+/* How a device executes a declared (weight, activation) pair (`enum Exec`). */
+typedef enum {
+    NVFP4_EXEC_FP4_MMA = 0,        /* block-scaled FP4 MMA: gemm_nvfp4_w4a4 */
+    NVFP4_EXEC_FP8_EXACT = 1,      /* exact E2M1->E4M3 conversion on the FP8 MMA: gemm_nvfp4_via_fp8 */
+    NVFP4_EXEC_BF16_WIDEN = 2,     /* BF16 MMA, NVFP4 weights widened in registers: gemm_w4a16 */
+    NVFP4_EXEC_NO_FP4_KERNEL = 3,  /* device has the FP4 MMA, but its class has no compiled kernel */
+    NVFP4_EXEC_NO_PATH = 4         /* neither native nor exact: refused, never widened */
+} nvfp4_exec;
+
+/* ---- planning (host only, no device work) -------------------------------- */
+
+/* kind_of: the MMA kind `activation` needs.  NVFP4_KIND_INVALID for a bad enum. */
+NVFP4_API nvfp4_kind nvfp4_kind_of(nvfp4_fmt activation);
+
+/* exec_of for a device CLASS given by its compute capability (e.g. 100 for
+ * sm_100, 90 for sm_90, 120 for sm_120).  Pure function; usable without a GPU.
+ * (NVFP4, NVFP4): FP4_MMA where this library compiles its block-scaled kernel
+ * for the class (sm_100 only), NO_FP4_KERNEL on other classes that have the
+ * FP4 MMA (sm_101/103/110/120/121), FP8_EXACT on a class without the FP4 MMA
+ * but with the FP8 MMA for which this library compiles the exact-path kernel
+ * (none besides sm_100, so NO_PATH on sm_89/sm_90), NO_PATH otherwise.
+ * (NVFP4, BF16): BF16_WIDEN on sm_100, NO_PATH elsewhere.
+ * (NVFP4, FP8) (W4A8): no single-instruction MMA; the exact E4M3 path, which
+ * this library does not carry yet, so NO_PATH.
+ * Pairs whose weights are not NVFP4: NO_PATH (this library carries NVFP4-weight
+ * paths only).  `fp4_kernel_disabled` != 0 behaves as if the class compiled no
+ * FP4 block-scale kernel (module doc, `fp4_fallback`, `avail::without_fp4_kernel`). */
+NVFP4_API nvfp4_exec nvfp4_exec_of_arch(int sm_arch, nvfp4_fmt weight, nvfp4_fmt activation,
+                              int fp4_kernel_disabled);
+
+/* exec_of for CUDA device `device` (queries its compute capability; NO_PATH if
+ * the device cannot be queried).  Honors nvfp4_set_fp4_kernel_disabled(). */
+NVFP4_API nvfp4_exec nvfp4_exec_of(int device, nvfp4_fmt weight, nvfp4_fmt activation);
+
+/* Process-wide switch that mimics a device class without a compiled FP4
+ * block-scale kernel (for planning tests): while set, exec_of reports
+ * NO_FP4_KERNEL for (NVFP4, NVFP4) and gemm_nvfp4_w4a4 / the grouped entry
+ * return NVFP4_ERR_NO_FP4_KERNEL without enqueueing anything. */
+NVFP4_API void nvfp4_set_fp4_kernel_disabled(int disabled);
+
+/* pair_name: the declared pair as "W4A16"-style text ("W4A4", "W4A8", "W16A16"
+ * ...).  Static storage; "?" for a bad enum. */
+NVFP4_API const char* nvfp4_pair_name(nvfp4_fmt weight, nvfp4_fmt activation);
+
+/* Human-readable name of an nvfp4_exec value (static storage). */
+NVFP4_API const char* nvfp4_exec_name(nvfp4_exec e);
+
+/* ---- matmuls --------------------------------------------------------------- */
+
+/* W4A4 on the block-scaled FP4 MMA (tcgen05.mma kind::mxf4nvf4, scale_vec::4X,
+ * E4M3 scales, FP32 accumulation in tensor memory, fused alpha and BF16
+ * epilogue).  M, N >= 0 (0 returns OK and does nothing); K >= 32, K % 32 == 0.
+ * Requires exec_of(device, NVFP4, NVFP4) == FP4_MMA, else NVFP4_ERR_NO_FP4_KERNEL
+ * or NVFP4_ERR_NOPATH. */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, float gA,
+                             const uint8_t* W, const uint8_t* sW, float gW,
+                             void* Y_bf16, int M, int N, int K, void* stream);
+
+/* The same product through the exact E2M1->E4M3 conversion on the FP8 MMA
+ * (module doc, bullet 2): each packed code byte is split into its two nibbles,
+ * each placed in the high nibble of a byte and converted by
+ * (q & 0x80808080) | ((q & 0x70707070) >> 2) to an E4M3 value equal to the
+ * code's value times 2^-6; each 16-group's FP8 partial sum is scaled in FP32 by
+ * (sA*2^6)*(sW*2^6) and accumulated.  Same arguments and preconditions as
+ * gemm_nvfp4_w4a4; needs a device class for which the FP8 kernel is compiled
+ * (sm_100), else NVFP4_ERR_NOPATH. */
+NVFP4_API nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, float gA,
+                                const uint8_t* W, const uint8_t* sW, float gW,
+                                void* Y_bf16, int M, int N, int K, void* stream);
+
+/* W4A16: BF16 activations A_bf16 [M][K] (row-major) times NVFP4 weights, the
+ * weights widened to BF16 in registers (exactly: an E2M1 value times an E4M3
+ * scale has at most 6 significant bits), FP32 accumulation, gW applied in the
+ * epilogue, BF16 output Y [M][N].  Memory-bound decode shape (small M).
+ * M >= 0, N >= 0, K >= 32, K % 32 == 0.  `workspace` must hold
+ * nvfp4_w4a16_workspace_size(M, N, K) bytes (device memory, 16-byte aligned;
+ * may be NULL when that size is 0); it holds FP32 split-K partial sums and
+ * is fully overwritten by every call (no zeroing needed). */
+NVFP4_API nvfp4_status gemm_w4a16(const void* A_bf16, const uint8_t* W, const uint8_t* sW, float gW,
+                        void* Y_bf16, int M, int N, int K,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace gemm_w4a16 needs for this shape on the current
+ * device (0 when the kernel runs without a split-K reduction). */
+NVFP4_API size_t nvfp4_w4a16_workspace_size(int M, int N, int K);
+
+/* Grouped (MoE) W4A4: expert e owns rows offsets[e] .. offsets[e+1]-1 of A
+ * (tokens grouped by expert), its weights W + e*N*K/2 ([N][K/2]), scales
+ * sW + e*N*K/16 ([N][K/16]) and FP32 scale gW_host[e].  Y is [offsets[E]][N].
+ * `offsets_host` (int32 [E+1], host memory, offsets[0] == 0, non-decreasing)
+ * is read during the call only.  Experts with fewer than 128 rows run with
+ * the operands swapped (Y_e^T = W_e . A_e^T: weight rows on the MMA's M side,
+ * tokens on its N side).  1 <= E <= 1024. */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t* A, const uint8_t* sA, float gA,
+                                     const uint8_t* W, const uint8_t* sW,
+                                     const float* gW_host, const int32_t* offsets_host,
+                                     int E, void* Y_bf16, int N, int K, void* stream);
+
+/* ---- diagnostics ----------------------------------------------------------- */
+
+/* Thread-local text of the last error returned on this host thread ("" if none). */
+NVFP4_API const char* nvfp4_last_error(void);
+
+/* Synchronizes `stream`, then reads and clears the device error word that a
+ * kernel sets when one of its bounded waits expires.  NVFP4_OK if clear,
+ * NVFP4_ERR_DEVICE_TIMEOUT if set, NVFP4_ERR_CUDA if synchronization failed. */
+NVFP4_API nvfp4_status nvfp4_check_device_error(void* stream);
+
+/* Library version string (static storage). */
+NVFP4_API const char* nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_B200_H */

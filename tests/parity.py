@@ -1,0 +1,33 @@
+"""Comparison rule shared by the GPU parity tests.
+
+Tolerance (from the matmul's specification): against the FP64 oracle value
+(not its BF16 rounding), relative Frobenius error <= 2e-3 and per-element
+|err| <= 1e-2 * max|ref|.  BF16 output rounding alone contributes ~1.5e-3 of
+relative Frobenius error; FP32 accumulation adds ~1e-6.  Guards against
+vacuous passes: the reference must be non-empty, finite and non-zero, the
+result finite, and both the same size.
+"""
+import numpy as np
+
+REL_FRO_TOL = 2e-3
+MAX_ABS_REL_TOL = 1e-2
+
+
+def bf16_to_f64(t) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check(y, ref, what=""):
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert y.shape == ref.shape, f"{what}: shape {y.shape} != {ref.shape}"
+    assert ref.size > 0, f"{what}: empty comparison"
+    assert np.all(np.isfinite(ref)), f"{what}: non-finite reference"
+    assert np.all(np.isfinite(y)), f"{what}: non-finite result ({np.sum(~np.isfinite(y))} values)"
+    nref = np.linalg.norm(ref)
+    assert nref > 0, f"{what}: all-zero reference"
+    rel = np.linalg.norm(y - ref) / nref
+    mx = np.max(np.abs(y - ref)) / np.max(np.abs(ref))
+    assert rel <= REL_FRO_TOL, f"{what}: relative Frobenius error {rel:.3e} > {REL_FRO_TOL}"
+    assert mx <= MAX_ABS_REL_TOL, f"{what}: max |err|/max|ref| {mx:.3e} > {MAX_ABS_REL_TOL}"
+    return rel, mx

@@ -1,0 +1,102 @@
+"""The C-ABI library: loads, exports every declared symbol, plans and rejects (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_scaled_precision_nvfp4_b200 as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^NVFP4_API\s+[\w\s\*]+?\b(\w+)\(", src, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = nv.load_library()
+    names = declared_functions()
+    assert len(names) >= 14
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in nv.C_FUNCTIONS, f"{name} has no binding"
+    assert set(nv.C_FUNCTIONS) == set(names)
+
+
+def test_library_is_sm100a_only_and_has_no_cpu_symbols():
+    # the product library carries no oracle code
+    lib = nv.load_library()
+    for bad in ("oracle_gemm_w4a4", "oracle_e2m1_value"):
+        with pytest.raises(AttributeError):
+            getattr(lib, bad)
+
+
+def test_kind_of():
+    assert nv.nvfp4_kind_of(nv.Fmt.BF16) == nv.Kind.BF16_MMA
+    assert nv.nvfp4_kind_of(nv.Fmt.FP8_E4M3) == nv.Kind.FP8_MMA
+    assert nv.nvfp4_kind_of(nv.Fmt.NVFP4) == nv.Kind.FP4_BLOCK_SCALED
+    assert nv.load_library().nvfp4_kind_of(7) == -1
+
+
+def test_pair_name():
+    F = nv.Fmt
+    assert nv.nvfp4_pair_name(F.NVFP4, F.NVFP4) == "W4A4"
+    assert nv.nvfp4_pair_name(F.NVFP4, F.BF16) == "W4A16"
+    assert nv.nvfp4_pair_name(F.NVFP4, F.FP8_E4M3) == "W4A8"
+    assert nv.nvfp4_pair_name(F.BF16, F.BF16) == "W16A16"
+    assert nv.load_library().nvfp4_pair_name(9, 0) == b"?"
+
+
+@pytest.mark.parametrize("arch,expect", [
+    (100, "FP4_MMA"), (103, "NO_FP4_KERNEL"), (120, "NO_FP4_KERNEL"), (90, "NO_PATH"),
+    (89, "NO_PATH"), (80, "NO_PATH")])
+def test_exec_of_w4a4_by_class(arch, expect):
+    assert nv.nvfp4_exec_of_arch(arch, nv.Fmt.NVFP4, nv.Fmt.NVFP4).name == expect
+
+
+def test_exec_of_other_pairs():
+    F, E = nv.Fmt, nv.Exec
+    assert nv.nvfp4_exec_of_arch(100, F.NVFP4, F.BF16) == E.BF16_WIDEN
+    assert nv.nvfp4_exec_of_arch(90, F.NVFP4, F.BF16) == E.NO_PATH
+    # W4A8: no single-instruction MMA; its exact path is not carried -> no path, never widened
+    assert nv.nvfp4_exec_of_arch(100, F.NVFP4, F.FP8_E4M3) == E.NO_PATH
+    for w in (F.BF16, F.FP8_E4M3):
+        for a in F:
+            assert nv.nvfp4_exec_of_arch(100, w, a) == E.NO_PATH
+
+
+def test_kernel_missing_flag_is_no_fp4_kernel_not_an_upcast():
+    E, F = nv.Exec, nv.Fmt
+    assert nv.nvfp4_exec_of_arch(100, F.NVFP4, F.NVFP4, fp4_kernel_disabled=True) \
+        == E.NO_FP4_KERNEL
+    # the activation format is never re-planned at a wider format
+    assert nv.nvfp4_exec_of_arch(90, F.NVFP4, F.NVFP4) != E.BF16_WIDEN
+
+
+def test_exec_of_without_device_is_no_path():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert nv.nvfp4_exec_of(0, nv.Fmt.NVFP4, nv.Fmt.NVFP4) == nv.Exec.NO_PATH
+
+
+def _call_w4a4(lib, A=16, sA=16, W=16, sW=16, Y=16, M=4, N=4, K=64, name="gemm_nvfp4_w4a4"):
+    return getattr(lib, name)(A, sA, 1.0, W, sW, 1.0, Y, M, N, K, None)
+
+
+@pytest.mark.parametrize("name", ["gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8"])
+def test_argument_errors_need_no_device(name):
+    lib = nv.load_library()
+    assert _call_w4a4(lib, M=-1, name=name) == nv.Status.INVALID_ARG
+    assert _call_w4a4(lib, K=48, name=name) == nv.Status.INVALID_ARG
+    assert _call_w4a4(lib, K=0, name=name) == nv.Status.INVALID_ARG
+    assert _call_w4a4(lib, A=0, name=name) == nv.Status.INVALID_ARG
+    assert _call_w4a4(lib, A=17, name=name) == nv.Status.MISALIGNED
+    assert _call_w4a4(lib, Y=24, name=name) == nv.Status.MISALIGNED
+    assert b"16-byte" in lib.nvfp4_last_error()
