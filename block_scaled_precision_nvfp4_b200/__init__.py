@@ -26,7 +26,7 @@ __all__ = [
     "nvfp4_kind_of", "nvfp4_exec_of", "nvfp4_exec_of_arch", "nvfp4_pair_name",
     "nvfp4_exec_name", "nvfp4_set_fp4_kernel_disabled", "nvfp4_version",
     "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_w4a16",
-    "nvfp4_w4a16_workspace_size", "gemm_nvfp4_w4a4_grouped", "C_FUNCTIONS",
+    "gemm_nvfp4_w4a4_grouped", "C_FUNCTIONS",
 ]
 
 
@@ -82,8 +82,7 @@ C_FUNCTIONS = {
     "nvfp4_check_device_error": (_I, [_P]),
     "gemm_nvfp4_w4a4": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_nvfp4_via_fp8": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
-    "gemm_w4a16": (_I, [_P, _P, _P, _F, _P, _I, _I, _I, _P, _Z, _P]),
-    "nvfp4_w4a16_workspace_size": (_Z, [_I, _I, _I]),
+    "gemm_w4a16": (_I, [_P, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_nvfp4_w4a4_grouped": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
 }
 
@@ -213,11 +212,7 @@ def gemm_nvfp4_via_fp8(A, sA, gA, W, sW, gW, out=None, stream=None):
     return _w4a4_common("gemm_nvfp4_via_fp8", A, sA, gA, W, sW, gW, out, stream)
 
 
-def nvfp4_w4a16_workspace_size(M: int, N: int, K: int) -> int:
-    return int(load_library().nvfp4_w4a16_workspace_size(int(M), int(N), int(K)))
-
-
-def gemm_w4a16(A, W, sW, gW, out=None, workspace=None, stream=None):
+def gemm_w4a16(A, W, sW, gW, out=None, stream=None):
     """Y[M,N] (bf16) = gW * A_bf16 . (W.sW)^T, weights widened to BF16 in registers."""
     torch = _torch()
     M, K = A.shape
@@ -228,13 +223,7 @@ def gemm_w4a16(A, W, sW, gW, out=None, workspace=None, stream=None):
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
-    need = nvfp4_w4a16_workspace_size(M, N, K)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=A.device)
-    pws = 0 if workspace is None else workspace.data_ptr()
-    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _err(load_library().gemm_w4a16(pa, pw, psw, float(gW), py, M, N, K, pws, wsb,
-                                   _stream_ptr(stream)))
+    _err(load_library().gemm_w4a16(pa, pw, psw, float(gW), py, M, N, K, _stream_ptr(stream)))
     return out
 
 

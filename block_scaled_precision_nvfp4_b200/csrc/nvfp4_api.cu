@@ -17,6 +17,7 @@
 #include "../../include/nvfp4.h"
 #include "ptx.cuh"
 #include "w4a4_kernel.cuh"
+#include "w4a16_kernel.cuh"
 
 namespace {
 
@@ -141,9 +142,10 @@ bool get_encoder() {
 }
 
 // 2D uint8 map over a row-major [rows][row_bytes] buffer, box [box_rows][box_bytes],
-// 128-byte swizzle (box_bytes must be 128), zero fill out of bounds.
+// zero fill out of bounds; 128-byte swizzle (box_bytes == 128) or none.
 nvfp4_status make_map_u8(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
-                         uint32_t box_bytes, uint32_t box_rows) {
+                         uint32_t box_bytes, uint32_t box_rows,
+                         CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     if (!get_encoder()) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint64_t dims[2] = {row_bytes, rows};
     cuuint64_t strides[1] = {row_bytes};
@@ -151,7 +153,7 @@ nvfp4_status make_map_u8(CUtensorMap* map, const void* base, uint64_t row_bytes,
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return NVFP4_OK;
@@ -268,25 +270,38 @@ nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, float gA, cons
 
     constexpr int BN = 256, STAGES = 4;
     using C = nvfp4::w4a4::Cfg<BN, STAGES>;
-    auto kern = nvfp4::w4a4::w4a4_kernel<BN, STAGES>;
-    CUtensorMap tmA, tmB;
+    const bool sf_tma = (K % nvfp4::w4a4::BK) == 0;  // scale row pitch K/16 is 16-byte aligned
+    auto kern = sf_tma ? nvfp4::w4a4::w4a4_kernel<BN, STAGES, true>
+                       : nvfp4::w4a4::w4a4_kernel<BN, STAGES, false>;
+    CUtensorMap tmA, tmB, tmSA, tmSB;
     if ((st = make_map_u8(&tmA, A, (uint64_t)K / 2, (uint64_t)M, nvfp4::w4a4::BKB,
                           nvfp4::w4a4::BM)) != NVFP4_OK)
         return st;
     if ((st = make_map_u8(&tmB, W, (uint64_t)K / 2, (uint64_t)N, nvfp4::w4a4::BKB, BN)) != NVFP4_OK)
         return st;
+    if (sf_tma) {
+        if ((st = make_map_u8(&tmSA, sA, (uint64_t)K / 16, (uint64_t)M, 16, nvfp4::w4a4::BM,
+                              CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+            return st;
+        if ((st = make_map_u8(&tmSB, sW, (uint64_t)K / 16, (uint64_t)N, 16, BN,
+                              CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+            return st;
+    } else {
+        tmSA = tmA;  // unused
+        tmSB = tmB;
+    }
     if ((st = set_smem(kern, C::SMEM_BYTES, info, "w4a4_kernel")) != NVFP4_OK) return st;
 
     const int tiles = ((M + nvfp4::w4a4::BM - 1) / nvfp4::w4a4::BM) * ((N + BN - 1) / BN);
     const int grid = tiles < info.num_sms ? tiles : info.num_sms;
     kern<<<grid, nvfp4::w4a4::NUM_THREADS, C::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
-        tmA, tmB, sA, sW, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
+        tmA, tmB, tmSA, tmSB, sA, sW, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launching w4a4_kernel");
     return ok();
 }
 
-// ------------------------------------------------------------------------- not yet built
+// ------------------------------------------------------------------------- via FP8
 nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, float, const uint8_t* W,
                                 const uint8_t* sW, float, void* Y, int M, int N, int K, void*) {
     nvfp4_status st = check_w4a4_args(A, sA, W, sW, Y, M, N, K);
@@ -294,12 +309,56 @@ nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, float, cons
     return fail(NVFP4_ERR_NOPATH, "gemm_nvfp4_via_fp8 is not built yet");
 }
 
-nvfp4_status gemm_w4a16(const void*, const uint8_t*, const uint8_t*, float, void*, int, int, int,
-                        void*, size_t, void*) {
-    return fail(NVFP4_ERR_NOPATH, "gemm_w4a16 is not built yet");
-}
+// ------------------------------------------------------------------------- W4A16
+nvfp4_status gemm_w4a16(const void* A, const uint8_t* W, const uint8_t* sW, float gW, void* Y,
+                        int M, int N, int K, void* stream) {
+    namespace k16 = nvfp4::w4a16;
+    if (M < 0 || N < 0) return fail(NVFP4_ERR_INVALID_ARG, "M and N must be >= 0 (got %d, %d)", M, N);
+    if (K < 32 || K % 32 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "K must be a positive multiple of 32 (got %d)", K);
+    if (M > 0 && N > 0) {
+        if (!A || !W || !sW || !Y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+        if (!aligned16(A) || !aligned16(W) || !aligned16(sW) || !aligned16(Y))
+            return fail(NVFP4_ERR_MISALIGNED, "every buffer must be 16-byte aligned");
+    }
+    int dev;
+    DevInfo info;
+    if (!current_device(dev, info)) return fail(NVFP4_ERR_CUDA, "cannot query the current CUDA device");
+    if (nvfp4_exec_of_arch(info.sm_arch, NVFP4_FMT_NVFP4, NVFP4_FMT_BF16, 0) != NVFP4_EXEC_BF16_WIDEN)
+        return fail(NVFP4_ERR_NOPATH, "W4A16 has no BF16-widen kernel for sm_%d", info.sm_arch);
+    if (M == 0 || N == 0) return ok();
 
-size_t nvfp4_w4a16_workspace_size(int, int, int) { return 0; }
+    const int total_spans = (K + k16::SPAN - 1) / k16::SPAN;
+    const int sps = (total_spans + k16::CLUSTER - 1) / k16::CLUSTER;
+    const size_t smem = k16::smem_bytes(sps);
+    nvfp4_status st = set_smem(k16::w4a16_kernel, smem, info, "w4a16_kernel");
+    if (st != NVFP4_OK) return st;
+    const int row_blocks = (N + 15) / 16;
+    const int clusters = (row_blocks + k16::WARPS - 1) / k16::WARPS;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(clusters * k16::CLUSTER);
+    cfg.blockDim = dim3(k16::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = k16::CLUSTER;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float out_scale = 128.0f * gW;  // undoes the 2^-7 carried by the widened weights
+    for (int m0 = 0; m0 < M; m0 += k16::TOK) {
+        const int mc = M - m0 < k16::TOK ? M - m0 : k16::TOK;
+        const uint16_t* a = static_cast<const uint16_t*>(A) + (size_t)m0 * K;
+        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y) + (size_t)m0 * N;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, k16::w4a16_kernel, a, W, sW, y, mc, N, K,
+                                           out_scale, sps);
+        if (e != cudaSuccess) return cuda_fail(e, "launching w4a16_kernel");
+    }
+    return ok();
+}
 
 nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t*, const uint8_t*, float, const uint8_t*,
                                      const uint8_t*, const float*, const int32_t*, int, void*, int,

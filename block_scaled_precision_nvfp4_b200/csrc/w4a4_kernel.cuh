@@ -5,16 +5,17 @@
 //
 // Design (one persistent CTA per SM, 12 warps):
 //   warp 0      TMA producer: 128-byte K-slices (256 codes) of the A and W
-//               tiles, 128-byte swizzle, into a STAGES-deep ring.
+//               tiles, 128-byte swizzle, into a STAGES-deep ring, and (when the
+//               scale row pitch allows) the matching raw [rows][16 B] scale tiles.
 //   warp 1      TMEM owner + MMA issuer (one thread): per stage copies the
 //               stage's scale factors smem -> TMEM (tcgen05.cp) and issues four
 //               tcgen05.mma kind::mxf4nvf4 scale_vec::4X (K = 64 each) into an
 //               FP32 accumulator in TMEM; commits free the stage.
-//   warp 2      scale-factor warp: reads the plain row-major E4M3 scales of the
-//               stage from global memory and writes them in the MMA's scale
-//               layout (per 128 rows and K = 64: 32 lines of 16 bytes, line i
-//               holding rows i, i+32, i+64, i+96) -- so callers pass plain
-//               [rows][K/16] scales and no reordering pass is needed.
+//   warp 2      scale-factor warp: rewrites the stage's plain row-major E4M3
+//               scales in place into the MMA's scale layout (per 128 rows and
+//               K = 64: 32 lines of 16 bytes, line i holding rows i, i+32, i+64,
+//               i+96), so callers pass plain [rows][K/16] scales and no
+//               reordering pass over global memory is needed.
 //   warps 4-11  epilogue: TMEM -> registers (tcgen05.ld), x alpha, BF16 RNE,
 //               stores to global; the accumulator is released as soon as it is
 //               in registers so the next tile's MMAs overlap the stores.
@@ -67,6 +68,7 @@ struct Cfg {
     static_assert(TMEM_USED <= 512, "TMEM budget exceeded");
     static constexpr uint32_t BYTES_A = BM * BKB;
     static constexpr uint32_t BYTES_B = BN * BKB;
+    static constexpr uint32_t BYTES_SF = (BM + BN) * 16;  // raw scale tiles per stage
     static constexpr size_t SMEM_BYTES = sizeof(Smem<BN, STAGES>) + 1024;
     __host__ __device__ static constexpr uint32_t sfa_col(int s) { return BN + s * (SFA_COLS + SFB_COLS); }
     __host__ __device__ static constexpr uint32_t sfb_col(int s) { return sfa_col(s) + SFA_COLS; }
@@ -112,9 +114,14 @@ __device__ __forceinline__ uint4 load_sf16(const uint8_t* __restrict__ s, int gr
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-template <int BN, int STAGES>
+// SF_TMA: the scale tiles arrive by TMA with the operand tiles (needs the scale
+// row pitch K/16 to be a multiple of 16 bytes, i.e. K % 256 == 0) and the
+// scale-factor warp only transposes them in shared memory; otherwise the
+// scale-factor warp reads them from global memory itself.
+template <int BN, int STAGES, bool SF_TMA>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+            const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
             const uint8_t* __restrict__ sA, const uint8_t* __restrict__ sW,
             __nv_bfloat16* __restrict__ Y, int M, int N, int K, float alpha) {
     using C = Cfg<BN, STAGES>;
@@ -145,6 +152,10 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         fence_mbarrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (SF_TMA) {
+            tma_prefetch_desc(&tmSA);
+            tma_prefetch_desc(&tmSB);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, C::TMEM_COLS);
@@ -166,9 +177,15 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!mbar_wait(&sm.empty[s], ph ^ 1, abort, ROLE_PRODUCER)) goto producer_done;
-                    mbar_arrive_expect_tx(&sm.tma_full[s], C::BYTES_A + C::BYTES_B);
+                    mbar_arrive_expect_tx(&sm.tma_full[s], C::BYTES_A + C::BYTES_B +
+                                                               (SF_TMA ? C::BYTES_SF : 0u));
                     tma_load_2d(sm.a[s], &tmA, &sm.tma_full[s], kb * BKB, mb * BM);
                     tma_load_2d(sm.b[s], &tmB, &sm.tma_full[s], kb * BKB, nb * BN);
+                    if (SF_TMA) {
+                        // raw [rows][16 B] scale tiles, transposed in place by warp 2
+                        tma_load_2d(sm.sfa[s], &tmSA, &sm.tma_full[s], kb * 16, mb * BM);
+                        tma_load_2d(sm.sfb[s], &tmSB, &sm.tma_full[s], kb * 16, nb * BN);
+                    }
                 }
             }
         producer_done:
@@ -231,6 +248,10 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------ scale factors
+        // Row rr of a 128-row block goes to word (rr%32)*4 + rr/32 of each
+        // k-step's 512-byte atom.  The lane -> row choice keeps the 32 stores of
+        // one instruction in 32 distinct banks and the 16-byte reads of each
+        // quarter-warp on 8 consecutive rows.
         const bool fast = (K % BK) == 0;
         int it = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
@@ -240,17 +261,28 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             for (int kb = 0; kb < num_kb; ++kb, ++it) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
-                if (!warp_wait(&sm.empty[s], ph ^ 1, abort, ROLE_SF)) { ok = false; break; }
-                // Row rr of a 128-row block goes to word (rr%32)*4 + rr/32 of each
-                // k-step's 512-byte atom.  Lane -> row choice keeps the 32 stores
-                // of one instruction in 32 distinct banks.
                 uint4 v[4 * (1 + NRB)];
+                if (SF_TMA) {
+                    if (!warp_wait(&sm.tma_full[s], ph, abort, ROLE_SF)) { ok = false; break; }
 #pragma unroll
-                for (int i = 0; i < 4 * (1 + NRB); ++i) {
-                    const int blk = i / 4;
-                    const int rr = 32 * (lane >> 3) + 8 * (i & 3) + (lane & 7);
-                    v[i] = blk == 0 ? load_sf16(sA, mb * BM + rr, M, kb, G, fast)
-                                    : load_sf16(sW, nb * BN + (blk - 1) * 128 + rr, N, kb, G, fast);
+                    for (int i = 0; i < 4 * (1 + NRB); ++i) {
+                        const int blk = i / 4;
+                        const int rr = 32 * (lane >> 3) + 8 * (i & 3) + (lane & 7);
+                        const uint4* raw = blk == 0
+                            ? reinterpret_cast<const uint4*>(sm.sfa[s]) + rr
+                            : reinterpret_cast<const uint4*>(sm.sfb[s]) + (blk - 1) * 128 + rr;
+                        v[i] = *raw;
+                    }
+                    __syncwarp();
+                } else {
+                    if (!warp_wait(&sm.empty[s], ph ^ 1, abort, ROLE_SF)) { ok = false; break; }
+#pragma unroll
+                    for (int i = 0; i < 4 * (1 + NRB); ++i) {
+                        const int blk = i / 4;
+                        const int rr = 32 * (lane >> 3) + 8 * (i & 3) + (lane & 7);
+                        v[i] = blk == 0 ? load_sf16(sA, mb * BM + rr, M, kb, G, fast)
+                                        : load_sf16(sW, nb * BN + (blk - 1) * 128 + rr, N, kb, G, fast);
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 4 * (1 + NRB); ++i) {

@@ -148,18 +148,13 @@ NVFP4_API nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, f
 /* W4A16: BF16 activations A_bf16 [M][K] (row-major) times NVFP4 weights, the
  * weights widened to BF16 in registers (exactly: an E2M1 value times an E4M3
  * scale has at most 6 significant bits), FP32 accumulation, gW applied in the
- * epilogue, BF16 output Y [M][N].  Memory-bound decode shape (small M).
- * M >= 0, N >= 0, K >= 32, K % 32 == 0.  `workspace` must hold
- * nvfp4_w4a16_workspace_size(M, N, K) bytes (device memory, 16-byte aligned;
- * may be NULL when that size is 0); it holds FP32 split-K partial sums and
- * is fully overwritten by every call (no zeroing needed). */
+ * epilogue, BF16 output Y [M][N].  Built for the memory-bound decode shape:
+ * one launch covers 16 tokens (larger M runs as consecutive 16-token launches,
+ * each re-reading W).  K is split across an 8-CTA cluster and the partial sums
+ * are reduced on chip in a fixed order, so the call needs no workspace and is
+ * deterministic.  M, N >= 0; K >= 32, K % 32 == 0. */
 NVFP4_API nvfp4_status gemm_w4a16(const void* A_bf16, const uint8_t* W, const uint8_t* sW, float gW,
-                        void* Y_bf16, int M, int N, int K,
-                        void* workspace, size_t workspace_bytes, void* stream);
-
-/* Bytes of device workspace gemm_w4a16 needs for this shape on the current
- * device (0 when the kernel runs without a split-K reduction). */
-NVFP4_API size_t nvfp4_w4a16_workspace_size(int M, int N, int K);
+                        void* Y_bf16, int M, int N, int K, void* stream);
 
 /* Grouped (MoE) W4A4: expert e owns rows offsets[e] .. offsets[e+1]-1 of A
  * (tokens grouped by expert), its weights W + e*N*K/2 ([N][K/2]), scales
