@@ -18,6 +18,7 @@
 #include "ptx.cuh"
 #include "w4a4_kernel.cuh"
 #include "w4a16_kernel.cuh"
+#include "via_fp8_kernel.cuh"
 
 namespace {
 
@@ -302,11 +303,39 @@ nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, float gA, cons
 }
 
 // ------------------------------------------------------------------------- via FP8
-nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, float, const uint8_t* W,
-                                const uint8_t* sW, float, void* Y, int M, int N, int K, void*) {
+nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, float gA, const uint8_t* W,
+                                const uint8_t* sW, float gW, void* Y, int M, int N, int K,
+                                void* stream) {
+    namespace v8 = nvfp4::via_fp8;
     nvfp4_status st = check_w4a4_args(A, sA, W, sW, Y, M, N, K);
     if (st != NVFP4_OK) return st;
-    return fail(NVFP4_ERR_NOPATH, "gemm_nvfp4_via_fp8 is not built yet");
+    if (K % v8::BK != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "the exact FP8 path needs K %% 256 == 0 (got %d)", K);
+    int dev;
+    DevInfo info;
+    if (!current_device(dev, info)) return fail(NVFP4_ERR_CUDA, "cannot query the current CUDA device");
+    if (!class_has_fp8_mma(info.sm_arch) || !class_compiles_fp8_exact_kernel(info.sm_arch))
+        return fail(NVFP4_ERR_NOPATH, "no exact FP8-path kernel is compiled for sm_%d", info.sm_arch);
+    if (M == 0 || N == 0) return ok();
+
+    CUtensorMap tmA, tmB, tmSA, tmSB;
+    if ((st = make_map_u8(&tmA, A, (uint64_t)K / 2, (uint64_t)M, 128, v8::BM)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmB, W, (uint64_t)K / 2, (uint64_t)N, 128, v8::BN)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmSA, sA, (uint64_t)K / 16, (uint64_t)M, 16, v8::BM,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_u8(&tmSB, sW, (uint64_t)K / 16, (uint64_t)N, 16, v8::BN,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+        return st;
+    if ((st = set_smem(v8::via_fp8_kernel, v8::SMEM_BYTES, info, "via_fp8_kernel")) != NVFP4_OK)
+        return st;
+    const int tiles = ((M + v8::BM - 1) / v8::BM) * ((N + v8::BN - 1) / v8::BN);
+    const int grid = tiles < info.num_sms ? tiles : info.num_sms;
+    v8::via_fp8_kernel<<<grid, v8::NUM_THREADS, v8::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
+        tmA, tmB, tmSA, tmSB, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launching via_fp8_kernel");
+    return ok();
 }
 
 // ------------------------------------------------------------------------- W4A16
