@@ -19,6 +19,7 @@
 #include "w4a4_kernel.cuh"
 #include "w4a16_kernel.cuh"
 #include "via_fp8_kernel.cuh"
+#include "grouped_kernel.cuh"
 
 namespace {
 
@@ -389,10 +390,68 @@ nvfp4_status gemm_w4a16(const void* A, const uint8_t* W, const uint8_t* sW, floa
     return ok();
 }
 
-nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t*, const uint8_t*, float, const uint8_t*,
-                                     const uint8_t*, const float*, const int32_t*, int, void*, int,
-                                     int, void*) {
-    return fail(NVFP4_ERR_NOPATH, "gemm_nvfp4_w4a4_grouped is not built yet");
+// ------------------------------------------------------------------------- grouped W4A4
+nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t* A, const uint8_t* sA, float gA,
+                                     const uint8_t* W, const uint8_t* sW, const float* gW_host,
+                                     const int32_t* offsets_host, int E, void* Y, int N, int K,
+                                     void* stream) {
+    namespace gk = nvfp4::grouped;
+    if (E < 1 || E > gk::MAX_EXPERTS)
+        return fail(NVFP4_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", gk::MAX_EXPERTS, E);
+    if (!offsets_host || !gW_host) return fail(NVFP4_ERR_INVALID_ARG, "null offsets or gW");
+    if (offsets_host[0] != 0) return fail(NVFP4_ERR_INVALID_ARG, "offsets[0] must be 0");
+    for (int e = 0; e < E; ++e)
+        if (offsets_host[e + 1] < offsets_host[e])
+            return fail(NVFP4_ERR_INVALID_ARG, "offsets must be non-decreasing");
+    const int M = offsets_host[E];
+    nvfp4_status st = check_w4a4_args(A, sA, W, sW, Y, M, N, K);
+    if (st != NVFP4_OK) return st;
+    if (K % gk::BK != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "the grouped path needs K %% 256 == 0 (got %d)", K);
+    if ((int64_t)E * N > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "E*N too large");
+    int dev;
+    DevInfo info;
+    if ((st = check_fp4_path(dev, info)) != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return ok();
+
+    gk::Params prm;
+    memset(&prm, 0, sizeof(prm));
+    prm.E = E;
+    prm.N = N;
+    prm.K = K;
+    int64_t total = 0;
+    for (int e = 0; e < E; ++e) {
+        prm.tile_start[e] = (int)total;
+        prm.row_start[e] = offsets_host[e];
+        prm.alpha[e] = gA * gW_host[e];
+        total += gk::tiles_of_expert(offsets_host[e + 1] - offsets_host[e], N);
+    }
+    if (total > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "too many tiles");
+    prm.tile_start[E] = (int)total;
+    prm.row_start[E] = M;
+
+    CUtensorMap tmA, tmW256, tmW128, tmSA, tmSW256, tmSW128;
+    const uint64_t wrows = (uint64_t)E * N;
+    if ((st = make_map_u8(&tmA, A, (uint64_t)K / 2, (uint64_t)M, gk::BKB, gk::BM)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmW256, W, (uint64_t)K / 2, wrows, gk::BKB, gk::BN)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmW128, W, (uint64_t)K / 2, wrows, gk::BKB, gk::SBN)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmSA, sA, (uint64_t)K / 16, (uint64_t)M, 16, gk::BM,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_u8(&tmSW256, sW, (uint64_t)K / 16, wrows, 16, gk::BN,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_u8(&tmSW128, sW, (uint64_t)K / 16, wrows, 16, gk::SBN,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+        return st;
+    if ((st = set_smem(gk::grouped_kernel, gk::C::SMEM_BYTES, info, "grouped_kernel")) != NVFP4_OK)
+        return st;
+    const int grid = total < info.num_sms ? (int)total : info.num_sms;
+    gk::grouped_kernel<<<grid, gk::NUM_THREADS, gk::C::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
+        tmA, tmW256, tmW128, tmSA, tmSW256, tmSW128, prm, reinterpret_cast<__nv_bfloat16*>(Y));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launching grouped_kernel");
+    return ok();
 }
 
 }  // extern "C"

@@ -100,3 +100,18 @@ def test_argument_errors_need_no_device(name):
     assert _call_w4a4(lib, A=17, name=name) == nv.Status.MISALIGNED
     assert _call_w4a4(lib, Y=24, name=name) == nv.Status.MISALIGNED
     assert b"16-byte" in lib.nvfp4_last_error()
+
+
+def test_grouped_argument_errors_need_no_device():
+    lib = nv.load_library()
+    gws = (ctypes.c_float * 3)(1.0, 1.0, 1.0)
+    def call(offs, E=2, K=256, N=64, A=16):
+        o = (ctypes.c_int32 * len(offs))(*offs)
+        return lib.gemm_nvfp4_w4a4_grouped(A, 16, 1.0, 16, 16, ctypes.cast(gws, ctypes.c_void_p),
+                                           ctypes.cast(o, ctypes.c_void_p), E, 16, N, K, None)
+    assert call([0, 6, 5]) == nv.Status.INVALID_ARG          # decreasing
+    assert call([1, 6, 8]) == nv.Status.INVALID_ARG          # offsets[0] != 0
+    assert call([0, 0], E=0) == nv.Status.INVALID_ARG        # no experts
+    assert call([0] * 3, E=300) == nv.Status.INVALID_ARG     # too many experts
+    assert call([0, 4, 8], K=96) == nv.Status.INVALID_ARG    # K % 32
+    assert call([0, 4, 8], A=24) == nv.Status.MISALIGNED
