@@ -3,7 +3,9 @@
 
 Workload: the FFN down projection, Y[4096,5376] = A[4096,14336] . W[5376,14336]^T
 in NVFP4 (two-level quantisation of N(0,1) activations and N(0,0.02) weights,
-seeded).  A step is one call of gemm_nvfp4_w4a4 on device-resident inputs.
+seeded).  A step packs the activations' scales into the MMA's layout
+(nvfp4_pack_scales) and runs gemm_nvfp4_w4a4_packed on device-resident inputs;
+the weights' scales are packed once, as at model load.
 L2 is flushed (a 256 MiB write) between timed steps, outside the timed events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -46,7 +48,7 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=["ffn_down", "tiny"], default="ffn_down")
+    p.add_argument("--workload", choices=list(WORKLOADS), default="ffn_down")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -62,11 +64,38 @@ def peaks():
         return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
 
 
+# Each workload: how to build it, which entry point a step calls, its algorithmic
+# work (flops) and bytes, and the roofline that bounds it.
+WORKLOADS = {
+    "ffn_down": dict(path="w4a4", bound="tensor", desc="FFN down W4A4 4096x5376x14336"),
+    "via_fp8": dict(path="via_fp8", bound="alu", desc="FFN down through the exact FP8 path"),
+    "w4a16": dict(path="w4a16", bound="hbm", desc="W4A16 decode 16x5376x14336"),
+    "grouped": dict(path="grouped", bound="tensor", desc="grouped MoE W4A4, 8 experts"),
+    "tiny": dict(path="w4a4", bound="tensor", desc="tiny W4A4 128x256x256"),
+}
+
+
 def make_workload(name):
     from block_scaled_precision_nvfp4_b200 import workloads as wl
     if name == "tiny":
         return wl.tiny_w4a4(0)
+    if name == "w4a16":
+        return wl.w4a16_decode()
+    if name == "grouped":
+        return wl.grouped_w4a4()
     return wl.ffn_down_w4a4()
+
+
+def algorithmic(wl_, path):
+    """(flops, bytes) of one step: 2*M*N*K and every input byte read once plus Y written."""
+    M, N, K = wl_.M, wl_.N, wl_.K
+    flops = 2.0 * M * N * K
+    ybytes = M * N * 2
+    if path == "w4a16":
+        return flops, N * K // 2 + N * K // 16 + M * K * 2 + ybytes
+    if path == "grouped":
+        return flops, wl_.E * (N * K // 2 + N * K // 16) + M * (K // 2 + K // 16) + ybytes
+    return flops, (M + N) * (K // 2 + K // 16) + ybytes
 
 
 # --- clock sampling during the timed region (NVML reads only) -------------------------
@@ -134,20 +163,34 @@ class ClockSampler:
 
 # --- the reference arm: the FP64 oracle on the host cores ------------------------------
 
-def oracle_rows_for(seconds, wl_, rate_probe_rows=4):
+def _oracle_rows(wl_, rows):
+    """The FP64 oracle on the first `rows` output rows of the workload."""
     import oracle
+    if wl_.A_bf16 is not None:
+        oracle.gemm_w4a16(wl_.A_bf16[:rows], wl_.W.codes, wl_.W.scales, wl_.W.g, rows, wl_.N,
+                          wl_.K)
+    elif wl_.E:
+        from block_scaled_precision_nvfp4_b200 import workloads as wlm
+        Wc, Ws, gW = wlm.stack_experts(wl_)
+        r = np.repeat(np.arange(rows), wl_.N)
+        c = np.tile(np.arange(wl_.N), rows)
+        oracle.gemm_grouped_w4a4(wl_.A.codes, wl_.A.scales, wl_.A.g, Wc, Ws,
+                                 gW.astype(np.float64), wl_.offsets, wl_.N, wl_.K, rows=r, cols=c)
+    else:
+        oracle.gemm_w4a4(wl_.A.codes[:rows], wl_.A.scales[:rows], wl_.A.g, wl_.W.codes,
+                         wl_.W.scales, wl_.W.g, rows, wl_.N, wl_.K)
+
+
+def oracle_rows_for(seconds, wl_, rate_probe_rows=2):
     t0 = time.perf_counter()
-    oracle.gemm_w4a4(wl_.A.codes[:rate_probe_rows], wl_.A.scales[:rate_probe_rows], wl_.A.g,
-                     wl_.W.codes, wl_.W.scales, wl_.W.g, rate_probe_rows, wl_.N, wl_.K)
+    _oracle_rows(wl_, rate_probe_rows)
     rate = rate_probe_rows / max(time.perf_counter() - t0, 1e-6)  # rows per second
     return int(max(1, min(wl_.M, round(rate * seconds))))
 
 
 def time_oracle(wl_, rows):
-    import oracle
     t0 = time.perf_counter()
-    oracle.gemm_w4a4(wl_.A.codes[:rows], wl_.A.scales[:rows], wl_.A.g, wl_.W.codes,
-                     wl_.W.scales, wl_.W.g, rows, wl_.N, wl_.K)
+    _oracle_rows(wl_, rows)
     dt = time.perf_counter() - t0
     return 2.0 * rows * wl_.N * wl_.K / dt / 1e12, dt
 
@@ -226,6 +269,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     import block_scaled_precision_nvfp4_b200 as nv
+    from block_scaled_precision_nvfp4_b200 import workloads as wlm
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -239,20 +283,55 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     nv.load_library(build_if_missing=False)
 
+    spec = WORKLOADS[args.workload]
+    path = spec["path"]
     wl_ = make_workload(args.workload)
     M, N, K = wl_.M, wl_.N, wl_.K
-    flops = 2.0 * M * N * K
+    flops, alg_bytes = algorithmic(wl_, path)
 
     def dev_(x):
         return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
 
-    A, sA, W, sW = dev_(wl_.A.codes), dev_(wl_.A.scales), dev_(wl_.W.codes), dev_(wl_.W.scales)
+    # host copies of the inputs (pinned) and their device twins
+    if path == "w4a16":
+        host = [wl_.A_bf16.view(np.int16), wl_.W.codes, wl_.W.scales]
+    elif path == "grouped":
+        Wc, Ws, gW = wlm.stack_experts(wl_)
+        host = [wl_.A.codes, wl_.A.scales, Wc, Ws]
+    else:
+        host = [wl_.A.codes, wl_.A.scales, wl_.W.codes, wl_.W.scales]
+    dv = [dev_(h) for h in host]
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        nv.gemm_nvfp4_w4a4(A, sA, wl_.A.g, W, sW, wl_.W.g, out=Y, stream=stream)
+    if path == "w4a16":
+        a16 = dv[0].view(torch.bfloat16)
+        def step():
+            nv.gemm_w4a16(a16, dv[1], dv[2], wl_.W.g, out=Y, stream=stream)
+    elif path == "grouped":
+        gw_list = [float(x) for x in gW]
+        offs = [int(x) for x in wl_.offsets]
+        def step():
+            nv.gemm_nvfp4_w4a4_grouped(dv[0], dv[1], wl_.A.g, dv[2], dv[3], gw_list, offs,
+                                       out=Y, stream=stream)
+    elif path == "via_fp8":
+        def step():
+            nv.gemm_nvfp4_via_fp8(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
+    else:
+        # W4A4: the weights' scales are packed once (model load); each step packs the
+        # activations' scales and runs the product on pairs of SMs.
+        sw_packed = nv.nvfp4_pack_scales(dv[3], K, stream=stream)
+        sa_packed = torch.empty(nv.nvfp4_scale_layout_bytes(M, K), dtype=torch.uint8, device=dev)
+        mid_events = []
+
+        def step(mid=None):
+            nv.nvfp4_pack_scales(dv[1], K, out=sa_packed, stream=stream)
+            if mid is not None:
+                mid.record(stream)
+            nv.gemm_nvfp4_w4a4_packed(dv[0], sa_packed, wl_.A.g, dv[2], sw_packed, wl_.W.g,
+                                      out=Y, stream=stream)
+    launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2}.get(path, 1)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -265,11 +344,15 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] if path == "w4a4" else None
     with ClockSampler(dev.index) as clk:
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
-            step()
+            if mids is not None:
+                step(mids[i])
+            else:
+                step()
             ends[i].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
@@ -286,14 +369,13 @@ def run_ours(args):
     # end to end through the public API: pinned host inputs -> device -> call -> host result
     e2e = None
     if not args.no_e2e:
-        hA, hsA, hW, hsW = (torch.from_numpy(np.ascontiguousarray(x)).pin_memory() for x in
-                            (wl_.A.codes, wl_.A.scales, wl_.W.codes, wl_.W.scales))
+        hp = [torch.from_numpy(np.ascontiguousarray(h)).pin_memory() for h in host]
         hY = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
         e_steps = max(1, min(args.steps, 20))
 
         def e2e_step():
-            A.copy_(hA, non_blocking=True); sA.copy_(hsA, non_blocking=True)
-            W.copy_(hW, non_blocking=True); sW.copy_(hsW, non_blocking=True)
+            for d, h in zip(dv, hp):
+                d.copy_(h, non_blocking=True)
             step()
             hY.copy_(Y, non_blocking=True)
 
@@ -313,31 +395,72 @@ def run_ours(args):
             tt = torch.tensor([te], dtype=torch.float64, device=dev)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             te = float(tt.item())
-        h2d = sum(x.numel() * x.element_size() for x in (hA, hsA, hW, hsW))
+        h2d = sum(x.numel() * x.element_size() for x in hp)
         e2e = {"value": world * flops / (te * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hY.numel() * 2,
                "ms_per_step": te}
 
-    bf16_peak, _, peak_src = peaks()
-    fp4_peak = bf16_peak * FP4_PER_BF16
-    achieved = flops / (t_ms * 1e-3) / 1e12
+    bf16_peak, hbm_peak, peak_src = peaks()
+    kern_s = t_ms * 1e-3
+    extra = {}
+    if mids is not None:
+        # the dominant kernel alone (the product), and the plain-scale entry point for context
+        gemm_ms = [m.elapsed_time(e) for m, e in zip(mids, ends)]
+        kern_s = (sum(gemm_ms) / len(gemm_ms)) * 1e-3
+        pack_ms = [s_.elapsed_time(m) for s_, m in zip(starts, mids)]
+        p0 = torch.cuda.Event(enable_timing=True); p1 = torch.cuda.Event(enable_timing=True)
+        plain = []
+        for _ in range(10):
+            flush.zero_()
+            p0.record(stream)
+            nv.gemm_nvfp4_w4a4(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
+            p1.record(stream)
+            torch.cuda.synchronize(dev)
+            plain.append(p0.elapsed_time(p1))
+        extra = {"pack_activation_scales_ms": statistics.median(pack_ms),
+                 "gemm_packed_ms": statistics.median(gemm_ms),
+                 "plain_scale_entry_ms": statistics.median(plain),
+                 "plain_scale_entry_tflops": flops / (statistics.median(plain) * 1e-3) / 1e12}
+    kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel",
+                   "w4a16": "w4a16_kernel", "grouped": "grouped_kernel"}[path]
+    if spec["bound"] == "tensor":
+        fp4_peak = bf16_peak * FP4_PER_BF16
+        achieved = flops / kern_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak,
+                "peak_note": f"{peak_src} bf16 {bf16_peak:.1f} TFLOP/s x nominal fp4/bf16 4"}
+    elif spec["bound"] == "hbm":
+        achieved = alg_bytes / kern_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "peak_note": f"{peak_src} copy bandwidth",
+                "algorithmic_bytes": alg_bytes}
+    else:
+        # one packed-f32x2 instruction per lane per (row, column, group) update:
+        # 148 SMs x 128 FP32 lanes x max clock
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        clk_mhz = clk.summary().get("sm_max_mhz") or 1965
+        peak_upd = sms * 128 * clk_mhz * 1e6 / 1e12  # T updates / s
+        achieved = (M * N * K / 16) / kern_s / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak_upd,
+                "unit": "Tupdate/s", "frac": achieved / peak_upd,
+                "peak_note": "per-16 FP32 scale-apply updates; derived: SMs x 128 lanes x max clock"}
+    roof.update({"traffic": profiled_traffic(wl_.name), "kernel": kernel_name,
+                 "kernel_ms": kern_s * 1e3})
+    roof.update(extra)
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "metric": METRIC if args.workload == "ffn_down" else f"{spec['desc']} TFLOP/s",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4(e2m1 x e2m1, e4m3 group scales) -> f32 accumulate -> bf16",
+        "dtype": ("bf16 x nvfp4(e2m1, e4m3 group scales) -> f32 accumulate -> bf16"
+                  if path == "w4a16" else
+                  "nvfp4(e2m1 x e2m1, e4m3 group scales) -> f32 accumulate -> bf16"),
         "data": "synthetic",
         "config": {"workload": wl_.name, "M": M, "N": N, "K": K, "global_batch": world * M,
                    "parallelism": f"dp{world}", "l2": "flushed between timed steps (256 MiB write)",
-                   "inputs": wl_.notes},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
-                     "unit": "TFLOP/s", "frac": achieved / fp4_peak,
-                     "peak_note": f"{peak_src} bf16 {bf16_peak:.1f} TFLOP/s x nominal fp4/bf16 4",
-                     "traffic": profiled_traffic(wl_.name),
-                     "kernel": "w4a4_kernel<256,4>",
-                     "per_launch_ms": {"median": statistics.median(per_step),
-                                       "min": min(per_step)}},
-        "gpu_launches": args.steps,
+                   "inputs": wl_.notes, "algorithmic_bytes": alg_bytes},
+        "roofline": roof,
+        "gpu_launches": args.steps * launches_per_step,
         "clocks": clk.summary(),
         "e2e": e2e,
     }

@@ -26,7 +26,8 @@ __all__ = [
     "nvfp4_kind_of", "nvfp4_exec_of", "nvfp4_exec_of_arch", "nvfp4_pair_name",
     "nvfp4_exec_name", "nvfp4_set_fp4_kernel_disabled", "nvfp4_version",
     "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_w4a16",
-    "gemm_nvfp4_w4a4_grouped", "C_FUNCTIONS",
+    "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
+    "gemm_nvfp4_w4a4_packed", "C_FUNCTIONS",
 ]
 
 
@@ -82,6 +83,9 @@ C_FUNCTIONS = {
     "nvfp4_check_device_error": (_I, [_P]),
     "gemm_nvfp4_w4a4": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_nvfp4_via_fp8": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
+    "nvfp4_scale_layout_bytes": (_Z, [_I, _I]),
+    "nvfp4_pack_scales": (_I, [_P, _I, _I, _P, _P]),
+    "gemm_nvfp4_w4a4_packed": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_w4a16": (_I, [_P, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_nvfp4_w4a4_grouped": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
 }
@@ -205,6 +209,47 @@ def _w4a4_common(fn_name, A, sA, gA, W, sW, gW, out, stream):
 def gemm_nvfp4_w4a4(A, sA, gA, W, sW, gW, out=None, stream=None):
     """Y[M,N] (bf16) = gA*gW * (A.sA)(W.sW)^T on the block-scaled FP4 MMA."""
     return _w4a4_common("gemm_nvfp4_w4a4", A, sA, gA, W, sW, gW, out, stream)
+
+
+def nvfp4_scale_layout_bytes(rows: int, K: int) -> int:
+    return int(load_library().nvfp4_scale_layout_bytes(int(rows), int(K)))
+
+
+def nvfp4_pack_scales(s, K=None, out=None, stream=None):
+    """Plain E4M3 scales uint8 [rows, K/16] -> the MMA's packed scale layout (uint8, 1-D)."""
+    torch = _torch()
+    rows, groups = s.shape
+    K = 16 * groups if K is None else int(K)
+    ps = _dev_tensor(s, torch.uint8, (rows, K // 16), "s")
+    n = nvfp4_scale_layout_bytes(rows, K)
+    if out is None:
+        out = torch.empty(max(n, 16), dtype=torch.uint8, device=s.device)
+    if out.dtype != torch.uint8 or not out.is_cuda or out.numel() < n or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous CUDA uint8 tensor of >= {n} bytes")
+    _err(load_library().nvfp4_pack_scales(ps, rows, K, out.data_ptr(), _stream_ptr(stream)))
+    return out
+
+
+def gemm_nvfp4_w4a4_packed(A, sA_packed, gA, W, sW_packed, gW, out=None, stream=None):
+    """gemm_nvfp4_w4a4 with scales packed by nvfp4_pack_scales (pairs of SMs, K % 256 == 0)."""
+    torch = _torch()
+    M, half_k = A.shape
+    N = W.shape[0]
+    K = 2 * half_k
+    pa = _dev_tensor(A, torch.uint8, (M, K // 2), "A")
+    pw = _dev_tensor(W, torch.uint8, (N, K // 2), "W")
+    for name, t, rows in (("sA_packed", sA_packed, M), ("sW_packed", sW_packed, N)):
+        need = nvfp4_scale_layout_bytes(rows, K)
+        if (not isinstance(t, torch.Tensor) or t.dtype != torch.uint8 or not t.is_cuda
+                or not t.is_contiguous() or t.numel() < need):
+            raise ValueError(f"{name} must be a contiguous CUDA uint8 tensor of >= {need} bytes")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
+    _err(load_library().gemm_nvfp4_w4a4_packed(pa, sA_packed.data_ptr(), float(gA), pw,
+                                               sW_packed.data_ptr(), float(gW), py, M, N, K,
+                                               _stream_ptr(stream)))
+    return out
 
 
 def gemm_nvfp4_via_fp8(A, sA, gA, W, sW, gW, out=None, stream=None):

@@ -17,6 +17,8 @@
 #include "../../include/nvfp4.h"
 #include "ptx.cuh"
 #include "w4a4_kernel.cuh"
+#include "w4a4_pair_kernel.cuh"
+#include "pack_scales_kernel.cuh"
 #include "w4a16_kernel.cuh"
 #include "via_fp8_kernel.cuh"
 #include "grouped_kernel.cuh"
@@ -161,6 +163,24 @@ nvfp4_status make_map_u8(CUtensorMap* map, const void* base, uint64_t row_bytes,
     return NVFP4_OK;
 }
 
+// 3D uint8 map over packed scales viewed as [blocks][ksteps*4][128 B]
+// (one 128-row block's packed scales are ksteps 512-byte atoms), box
+// (128, 16, box_blocks): one K-block (four K = 64 steps) of box_blocks blocks.
+nvfp4_status make_map_packed_sf(CUtensorMap* map, const void* base, uint64_t blocks,
+                                uint64_t ksteps, uint32_t box_blocks) {
+    if (!get_encoder()) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[3] = {128, ksteps * 4, blocks};
+    cuuint64_t strides[2] = {128, ksteps * 512};
+    cuuint32_t box[3] = {128, 16, box_blocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return NVFP4_OK;
+}
+
 // ---------------------------------------------------------------- argument checks
 nvfp4_status check_w4a4_args(const void* A, const void* sA, const void* W, const void* sW,
                              const void* Y, int M, int N, int K) {
@@ -270,9 +290,9 @@ nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, float gA, cons
     if ((st = check_fp4_path(dev, info)) != NVFP4_OK) return st;
     if (M == 0 || N == 0) return ok();
 
+    const bool sf_tma = (K % nvfp4::w4a4::BK) == 0;  // scale row pitch K/16 is 16-byte aligned
     constexpr int BN = 256, STAGES = 4;
     using C = nvfp4::w4a4::Cfg<BN, STAGES>;
-    const bool sf_tma = (K % nvfp4::w4a4::BK) == 0;  // scale row pitch K/16 is 16-byte aligned
     auto kern = sf_tma ? nvfp4::w4a4::w4a4_kernel<BN, STAGES, true>
                        : nvfp4::w4a4::w4a4_kernel<BN, STAGES, false>;
     CUtensorMap tmA, tmB, tmSA, tmSB;
@@ -300,6 +320,76 @@ nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, float gA, cons
         tmA, tmB, tmSA, tmSB, sA, sW, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launching w4a4_kernel");
+    return ok();
+}
+
+// ------------------------------------------------------------------------- packed scales
+size_t nvfp4_scale_layout_bytes(int rows, int K) {
+    if (rows < 0 || K < 64 || K % 64 != 0) return 0;
+    return (size_t)((rows + 127) / 128) * 128 * (size_t)(K / 16);
+}
+
+nvfp4_status nvfp4_pack_scales(const uint8_t* s_plain, int rows, int K, uint8_t* s_packed,
+                               void* stream) {
+    if (rows < 0) return fail(NVFP4_ERR_INVALID_ARG, "rows must be >= 0 (got %d)", rows);
+    if (K < 64 || K % 64 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "packing needs K %% 64 == 0 (got %d)", K);
+    if (rows == 0) return ok();
+    if (!s_plain || !s_packed) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(s_packed)) return fail(NVFP4_ERR_MISALIGNED, "s_packed must be 16-byte aligned");
+    const long long lines = (long long)((rows + 127) / 128) * (K / 64) * 32;
+    const int threads = 256;
+    const long long blocks = (lines + threads - 1) / threads;
+    if (blocks > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "scale matrix too large");
+    nvfp4::pack::pack_scales_kernel<<<(unsigned)blocks, threads, 0,
+                                      static_cast<cudaStream_t>(stream)>>>(
+        s_plain, s_packed, rows, K / 16, K / 64, lines);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launching pack_scales_kernel");
+    return ok();
+}
+
+nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, float gA,
+                                    const uint8_t* W, const uint8_t* sW_packed, float gW,
+                                    void* Y, int M, int N, int K, void* stream) {
+    namespace wp = nvfp4::w4a4_pair;
+    nvfp4_status st = check_w4a4_args(A, sA_packed, W, sW_packed, Y, M, N, K);
+    if (st != NVFP4_OK) return st;
+    if (K % wp::BK != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "the packed-scale path needs K %% 256 == 0 (got %d)", K);
+    int dev;
+    DevInfo info;
+    if ((st = check_fp4_path(dev, info)) != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return ok();
+    if (info.num_sms < 2) return fail(NVFP4_ERR_CUDA, "the pair kernel needs at least two SMs");
+
+    CUtensorMap tmA, tmB, tmSA, tmSB;
+    const uint64_t ks = (uint64_t)K / 64;
+    if ((st = make_map_u8(&tmA, A, (uint64_t)K / 2, (uint64_t)M, wp::BKB, wp::BM)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmB, W, (uint64_t)K / 2, (uint64_t)N, wp::BKB, wp::BNH)) != NVFP4_OK) return st;
+    if ((st = make_map_packed_sf(&tmSA, sA_packed, (uint64_t)(M + 127) / 128, ks, 1)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_packed_sf(&tmSB, sW_packed, (uint64_t)(N + 127) / 128, ks, wp::NRB)) != NVFP4_OK)
+        return st;
+    if ((st = set_smem(wp::w4a4_pair_kernel, wp::SMEM_BYTES, info, "w4a4_pair_kernel")) != NVFP4_OK)
+        return st;
+    const int tiles = ((M + wp::TILE_M - 1) / wp::TILE_M) * ((N + wp::BN - 1) / wp::BN);
+    const int pairs = tiles < info.num_sms / 2 ? tiles : info.num_sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(wp::NUM_THREADS);
+    cfg.dynamicSmemBytes = wp::SMEM_BYTES;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, wp::w4a4_pair_kernel, tmA, tmB, tmSA, tmSB,
+                                       reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
+    if (e != cudaSuccess) return cuda_fail(e, "launching w4a4_pair_kernel");
     return ok();
 }
 
@@ -363,6 +453,8 @@ nvfp4_status gemm_w4a16(const void* A, const uint8_t* W, const uint8_t* sW, floa
     const size_t smem = k16::smem_bytes(sps);
     nvfp4_status st = set_smem(k16::w4a16_kernel, smem, info, "w4a16_kernel");
     if (st != NVFP4_OK) return st;
+    // the whole unified L1/shared array as shared memory: three CTAs per SM
+    cudaFuncSetAttribute(k16::w4a16_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     const int row_blocks = (N + 15) / 16;
     const int clusters = (row_blocks + k16::WARPS - 1) / k16::WARPS;
 

@@ -7,7 +7,9 @@
 //   warp 0      TMA producer: 128-byte K-slices (256 codes) of the A and W
 //               tiles, 128-byte swizzle, into a STAGES-deep ring, and (when the
 //               scale row pitch allows) the matching raw [rows][16 B] scale tiles.
-//   warp 1      TMEM owner + MMA issuer (one thread): per stage copies the
+//   warp 1      TMEM owner + MMA issuer (one elected lane of the converged
+//               warp -- a warp that issues tcgen05 work keeps its lanes
+//               together instead of parking 31 of them): per stage copies the
 //               stage's scale factors smem -> TMEM (tcgen05.cp) and issues four
 //               tcgen05.mma kind::mxf4nvf4 scale_vec::4X (K = 64 each) into an
 //               FP32 accumulator in TMEM; commits free the stage.
@@ -93,10 +95,10 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 
 // Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int role) {
+                                          int role, uint32_t backoff_ns = 0) {
     const int lane = threadIdx.x & 31;
     int ok = 1;
-    if (lane == 0) ok = mbar_wait(bar, parity, abort, role) ? 1 : 0;
+    if (lane == 0) ok = mbar_wait(bar, parity, abort, role, backoff_ns) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -168,15 +170,17 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int it = 0;
-            for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
-                int mb, nb;
-                tile_coords(tile, num_m, num_n, mb, nb);
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1, abort, ROLE_PRODUCER)) goto producer_done;
+        // The whole warp walks the loop (converged); one elected lane issues.
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!warp_wait(&sm.empty[s], ph ^ 1, abort, ROLE_PRODUCER)) { ok = false; break; }
+                if (elect_one()) {
                     mbar_arrive_expect_tx(&sm.tma_full[s], C::BYTES_A + C::BYTES_B +
                                                                (SF_TMA ? C::BYTES_SF : 0u));
                     tma_load_2d(sm.a[s], &tmA, &sm.tma_full[s], kb * BKB, mb * BM);
@@ -187,34 +191,36 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                         tma_load_2d(sm.sfb[s], &tmSB, &sm.tma_full[s], kb * 16, nb * BN);
                     }
                 }
+                __syncwarp();
             }
-        producer_done:
-            if (*abort) {
-                // Let every copy this thread started land before the CTA exits.
-                for (int j = max(0, it - STAGES); j < it; ++j) {
-                    uint64_t* bar = &sm.tma_full[j % STAGES];
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(bar, (j / STAGES) & 1) &&
-                           globaltimer_ns() - t0 < kWaitLimitNs) {
-                    }
+        }
+        if (!ok && lane == 0) {
+            // Let every copy this warp started land before the CTA exits.
+            for (int j = max(0, it - STAGES); j < it; ++j) {
+                uint64_t* bar = &sm.tma_full[j % STAGES];
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(bar, (j / STAGES) & 1) && globaltimer_ns() - t0 < kWaitLimitNs) {
                 }
             }
         }
+        __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_mxf4nvf4(BM, BN);
-            int it = 0, tc = 0;
-            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
-                if (!mbar_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) break;
+        // Converged warp; the elected lane (the same lane every time) issues the
+        // scale copies, the MMAs and the commits that track them.
+        const uint32_t idesc = idesc_mxf4nvf4(BM, BN);
+        int it = 0, tc = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
+            if (!warp_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
+            tc_fence_after();
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!warp_wait(&sm.tma_full[s], ph, abort, ROLE_MMA) ||
+                    !warp_wait(&sm.sf_full[s], ph, abort, ROLE_MMA)) { ok = false; break; }
                 tc_fence_after();
-                bool ok = true;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(&sm.tma_full[s], ph, abort, ROLE_MMA) ||
-                        !mbar_wait(&sm.sf_full[s], ph, abort, ROLE_MMA)) { ok = false; break; }
-                    tc_fence_after();
+                if (elect_one()) {
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks)
                         tmem_cp_32x128b_x4(tmem + C::sfa_col(s) + ks * 4,
@@ -233,10 +239,14 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                                      tmem + C::sfb_col(s) + ks * NRB * 4, (kb | ks) != 0);
                     mma_commit(&sm.empty[s]);
                 }
-                if (!ok) break;
-                mma_commit(&sm.acc_full);
+                __syncwarp();
             }
-            // Wait for every MMA and copy this thread issued before TMEM is freed.
+            if (!ok) break;
+            if (elect_one()) mma_commit(&sm.acc_full);
+            __syncwarp();
+        }
+        // Every MMA and copy issued completes before TMEM is freed.
+        if (elect_one()) {
             mma_commit(&sm.drain);
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&sm.drain, 0)) {
@@ -246,6 +256,7 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                 }
             }
         }
+        __syncwarp();
     } else if (warp == 2) {
         // ------------------------------------------------------------ scale factors
         // Row rr of a 128-row block goes to word (rr%32)*4 + rr/32 of each

@@ -1,0 +1,279 @@
+// w4a4_pair_kernel.cuh -- NVFP4 W4A4 matmul on pairs of SMs (tcgen05 cta_group::2)
+// with scales already in the MMA's scale layout (pack_scales_kernel.cuh).
+//
+// Same product as w4a4_kernel.cuh (metrale_circuit `hardware::exec` module doc,
+// bullet 1, the NVFP4 row), with 256 x 256 output tiles computed by a cluster
+// of two CTAs on two SMs:
+//   * each CTA loads, with plain TMA tile loads, its own 128 rows of A, its own
+//     128 rows of W (half of the tile's N), the packed scales of its A rows and
+//     the packed scales of all 256 W rows; completion of both CTAs' loads is
+//     counted on one barrier in the leader CTA (rank 0), armed for both;
+//   * the leader's MMA thread copies both CTAs' scales to their TMEM
+//     (tcgen05.cp.cta_group::2: one instruction serves both SMs) and issues
+//     tcgen05.mma.cta_group::2 kind::mxf4nvf4 M=256 N=256 K=64; its commits
+//     free the stage in both CTAs;
+//   * each CTA's epilogue reads its own 128 x 256 accumulator.
+// Against one SM per 128 x 256 tile, every SM reads half as many W bytes per
+// flop and the pair issues half as many scale copies per flop; with the
+// scales packed ahead there is no shared-memory rewrite or cross-CTA hand-off
+// on the critical path.  All waits are bounded; both CTAs meet at a cluster
+// barrier before the pair's TMEM is freed.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "w4a4_kernel.cuh"
+
+namespace nvfp4 {
+namespace w4a4_pair {
+
+using w4a4::BK;
+using w4a4::BKB;
+using w4a4::KSTEPS;
+using w4a4::ROLE_DRAIN;
+using w4a4::ROLE_EPI;
+using w4a4::ROLE_MMA;
+using w4a4::ROLE_PRODUCER;
+using w4a4::warp_wait;
+
+constexpr int BM = 128;        // rows of A per CTA (the pair covers 256)
+constexpr int TILE_M = 256;
+constexpr int BN = 256;        // tile columns (rows of W) per pair
+constexpr int BNH = 128;       // rows of W loaded by each CTA
+constexpr int NRB = BN / 128;  // 128-row scale blocks of W per tile
+constexpr int STAGES = 5;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS);
+constexpr int FIRST_EPI_WARP = 2;
+constexpr int GROUP_M = 8;
+
+struct Smem {
+    alignas(1024) uint8_t a[STAGES][BM * BKB];
+    alignas(1024) uint8_t b[STAGES][BNH * BKB];
+    alignas(128) uint32_t sfa[STAGES][KSTEPS * 128];        // [ks][512-byte atom]
+    alignas(128) uint32_t sfb[STAGES][NRB * KSTEPS * 128];  // [rb][ks][512-byte atom]
+    uint64_t full[STAGES];   // leader: every byte of the stage, both CTAs
+    uint64_t empty[STAGES];  // each CTA: stage free (commit from the leader)
+    uint64_t acc_full;       // each CTA: accumulator ready (commit from the leader)
+    uint64_t acc_empty;      // leader: both CTAs' epilogues have read TMEM
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// one CTA's bytes per stage: A, half of W, sA of its rows, sW of all 256 rows
+constexpr uint32_t BYTES_CTA = (BM + BNH) * BKB + (BM + BN) * 16;
+constexpr int SFA_COLS = KSTEPS * 4, SFB_COLS = KSTEPS * NRB * 4;
+constexpr int TMEM_COLS = 512;
+static_assert(BN + STAGES * (SFA_COLS + SFB_COLS) <= TMEM_COLS, "TMEM budget exceeded");
+constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
+__host__ __device__ constexpr uint32_t sfa_col(int s) { return BN + s * (SFA_COLS + SFB_COLS); }
+__host__ __device__ constexpr uint32_t sfb_col(int s) { return sfa_col(s) + SFA_COLS; }
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
+    const int per_group = GROUP_M * num_n;
+    const int first_m = (tile / per_group) * GROUP_M;
+    const int gsize = min(num_m - first_m, GROUP_M);
+    const int in_group = tile % per_group;
+    mb = first_m + in_group % gsize;
+    nb = in_group / gsize;
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int32_t x, int32_t y,
+                                                 int32_t z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster),
+          "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 B x 128 rows
+                 const __grid_constant__ CUtensorMap tmB,   // W codes, box 128 B x 128 rows
+                 const __grid_constant__ CUtensorMap tmSA,  // packed sA: [rb][ks*4][128 B], box (128, 16, 1)
+                 const __grid_constant__ CUtensorMap tmSB,  // packed sW: same view, box (128, 16, 2)
+                 __nv_bfloat16* __restrict__ Y, int M, int N, int K, float alpha) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                        ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cid = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const int num_m = (M + TILE_M - 1) / TILE_M, num_n = (N + BN - 1) / BN;
+    const int tiles = num_m * num_n;
+    const int num_kb = K / BK;
+    volatile int* abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.acc_empty, 2 * NUM_EPI_WARPS);
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmSA);
+        tma_prefetch_desc(&tmSB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&sm.tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        int it = 0;
+        bool ok = true;
+        for (int tile = cid; tile < tiles && ok; tile += nclusters) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            const int arb = mb * 2 + (int)rank;  // this CTA's 128-row block of A
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % STAGES;
+                if (!warp_wait(&sm.empty[s], ((it / STAGES) & 1) ^ 1, abort, ROLE_PRODUCER, 32)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
+                    if (leader) mbar_arrive_expect_tx(&sm.full[s], 2 * BYTES_CTA);
+                    const uint32_t full0 = map_to_rank(&sm.full[s], 0);
+                    tma_load_2d_pair(sm.a[s], &tmA, full0, kb * BKB, arb * BM);
+                    tma_load_2d_pair(sm.b[s], &tmB, full0, kb * BKB, nb * BN + (int)rank * BNH);
+                    tma_load_3d_pair(sm.sfa[s], &tmSA, full0, 0, kb * 16, arb);
+                    tma_load_3d_pair(sm.sfb[s], &tmSB, full0, 0, kb * 16, nb * NRB);
+                }
+                __syncwarp();
+            }
+        }
+        if (!ok && leader && lane == 0) {
+            // every copy of this pair lands before either CTA leaves
+            for (int j = max(0, it - STAGES); j < it; ++j) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&sm.full[j % STAGES], (j / STAGES) & 1) &&
+                       globaltimer_ns() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (leader) {
+            const uint32_t idesc = idesc_mxf4nvf4(TILE_M, BN);
+            int it = 0, tc = 0;
+            bool ok = true;
+            for (int tile = cid; tile < tiles && ok; tile += nclusters, ++tc) {
+                if (!warp_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (!warp_wait(&sm.full[s], (it / STAGES) & 1, abort, ROLE_MMA)) { ok = false; break; }
+                    tc_fence_after();
+                    if (elect_one()) {
+#pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks)
+                            tmem_cp_32x128b_x4_pair(tmem + sfa_col(s) + ks * 4,
+                                                    desc_sf_32x16(smem_u32(&sm.sfa[s][ks * 128])));
+#pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+                            for (int rb = 0; rb < NRB; ++rb)
+                                tmem_cp_32x128b_x4_pair(
+                                    tmem + sfb_col(s) + (ks * NRB + rb) * 4,
+                                    desc_sf_32x16(smem_u32(&sm.sfb[s][(rb * KSTEPS + ks) * 128])));
+                        const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+#pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks)
+                            mma_mxf4nvf4_pair(tmem, desc_kmajor_sw128(a0 + ks * 32),
+                                              desc_kmajor_sw128(b0 + ks * 32), idesc,
+                                              tmem + sfa_col(s) + ks * 4,
+                                              tmem + sfb_col(s) + ks * NRB * 4, (kb | ks) != 0);
+                        mma_commit_pair(&sm.empty[s], 0x3);
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (elect_one()) mma_commit_pair(&sm.acc_full, 0x3);
+                __syncwarp();
+            }
+            if (elect_one()) {
+                mma_commit_pair(&sm.drain, 0x1);
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&sm.drain, 0)) {
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        atomicOr(&g_device_error, 1 | (ROLE_DRAIN << 8));
+                        break;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3, half = (warp - FIRST_EPI_WARP) >> 2;
+        constexpr int COLS = BN / 2, CHUNKS = COLS / 32;
+        const bool vec_ok = (N % 8) == 0;
+        int tc = 0;
+        for (int tile = cid; tile < tiles; tile += nclusters, ++tc) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI, 256)) break;
+            tc_fence_after();
+            uint32_t packed[COLS / 2];
+#pragma unroll
+            for (int c = 0; c < CHUNKS; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + half * COLS + c * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
+                                                             __uint_as_float(r[2 * j + 1]) * alpha);
+                    packed[c * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(&sm.acc_empty, 0);
+
+            const int row = mb * TILE_M + (int)rank * BM + 32 * q + lane;
+            const int col0 = nb * BN + half * COLS;
+            if (row < M) {
+                __nv_bfloat16* yrow = Y + (size_t)row * N;
+                if (vec_ok && col0 + COLS <= N) {
+                    uint4* dst = reinterpret_cast<uint4*>(yrow + col0);
+#pragma unroll
+                    for (int j = 0; j < COLS / 8; ++j)
+                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                            packed[4 * j + 3]);
+                } else {
+                    uint16_t* y16 = reinterpret_cast<uint16_t*>(yrow);
+#pragma unroll
+                    for (int j = 0; j < COLS; ++j)
+                        if (col0 + j < N) y16[col0 + j] = (uint16_t)(packed[j >> 1] >> (16 * (j & 1)));
+                }
+            }
+        }
+    }
+
+    // No CTA of the pair leaves (or frees TMEM) while the other may still use it.
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem, TMEM_COLS);
+}
+
+}  // namespace w4a4_pair
+}  // namespace nvfp4

@@ -133,6 +133,33 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, floa
                              const uint8_t* W, const uint8_t* sW, float gW,
                              void* Y_bf16, int M, int N, int K, void* stream);
 
+/* ---- scales in the MMA's layout ------------------------------------------- */
+
+/* Bytes of a packed scale buffer for a [rows][K/16] scale matrix (0 if K is
+ * not a positive multiple of 64): ceil(rows/128) * 128 * K/16. */
+NVFP4_API size_t nvfp4_scale_layout_bytes(int rows, int K);
+
+/* Rearranges plain E4M3 group scales s_plain [rows][K/16] (device, row-major)
+ * into the block-scaled MMA's scale layout in s_packed (device, 16-byte
+ * aligned, nvfp4_scale_layout_bytes(rows, K) bytes, caller-owned):
+ *     s_packed[rb][ks][i][j][t] = s_plain[rb*128 + 32*j + i][4*ks + t]
+ * for 128-row blocks rb, K = 64 steps ks, i < 32, j < 4, t < 4 (rows past
+ * `rows` are zero).  One 512-byte [i][j][t] atom is exactly what one
+ * tcgen05.cp 32x128b.warpx4 copies into TMEM for 128 rows and one K = 64 step.
+ * Weights' scales are packed once; activations' scales once per product.
+ * K % 64 == 0.  Asynchronous on `stream`. */
+NVFP4_API nvfp4_status nvfp4_pack_scales(const uint8_t* s_plain, int rows, int K,
+                                         uint8_t* s_packed, void* stream);
+
+/* gemm_nvfp4_w4a4 with both scale matrices already packed
+ * (nvfp4_pack_scales).  Runs on pairs of SMs (tcgen05 cta_group::2, 256 x 256
+ * tiles) and moves the packed scales with plain TMA tile loads, so no scale
+ * rewrite happens inside the product.  Same operation, operands and errors as
+ * gemm_nvfp4_w4a4, with K % 256 == 0. */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, float gA,
+                                              const uint8_t* W, const uint8_t* sW_packed, float gW,
+                                              void* Y_bf16, int M, int N, int K, void* stream);
+
 /* The same product through the exact E2M1->E4M3 conversion on the FP8 MMA
  * (module doc, bullet 2): each packed code byte is split into its two nibbles,
  * each placed in the high nibble of a byte and converted by

@@ -22,7 +22,7 @@ def declared_functions():
 def test_library_exports_every_declared_symbol():
     lib = nv.load_library()
     names = declared_functions()
-    assert len(names) >= 13
+    assert len(names) >= 16
     for name in names:
         assert hasattr(lib, name), name
         assert name in nv.C_FUNCTIONS, f"{name} has no binding"
