@@ -238,27 +238,36 @@ def run_reference(args):
 
 # --- our arm ---------------------------------------------------------------------------
 
-def kernel_source_hash():
+# the sources that define each workload's dominant kernel (the stored ncu traffic
+# of a kernel is used only while these are unchanged)
+KERNEL_SOURCES = {
+    "w4a4": ["w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
+    "via_fp8": ["via_fp8_kernel.cuh", "ptx.cuh"],
+    "w4a16": ["w4a16_kernel.cuh"],
+    "grouped": ["grouped_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
+}
+
+
+def kernel_source_hash(path):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_scaled_precision_nvfp4_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(f.read())
+    for n in KERNEL_SOURCES[path]:
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload_name):
+def profiled_traffic(workload_name, path):
     """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
-    path = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.txt")
+    fn = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.txt")
     try:
         kv = {}
-        with open(path) as f:
+        with open(fn) as f:
             for ln in f:
                 if ":" in ln:
                     k, v = ln.split(":", 1)
                     kv[k.strip()] = v.strip()
-        if kv.get("source_hash") == kernel_source_hash():
+        if kv.get("source_hash") == kernel_source_hash(path):
             return float(kv["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -444,7 +453,7 @@ def run_ours(args):
         roof = {"bound": "alu", "achieved": achieved, "peak": peak_upd,
                 "unit": "Tupdate/s", "frac": achieved / peak_upd,
                 "peak_note": "per-16 FP32 scale-apply updates; derived: SMs x 128 lanes x max clock"}
-    roof.update({"traffic": profiled_traffic(wl_.name), "kernel": kernel_name,
+    roof.update({"traffic": profiled_traffic(wl_.name, path), "kernel": kernel_name,
                  "kernel_ms": kern_s * 1e3})
     roof.update(extra)
     line = {

@@ -336,14 +336,14 @@ nvfp4_status nvfp4_pack_scales(const uint8_t* s_plain, int rows, int K, uint8_t*
         return fail(NVFP4_ERR_INVALID_ARG, "packing needs K %% 64 == 0 (got %d)", K);
     if (rows == 0) return ok();
     if (!s_plain || !s_packed) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
-    if (!aligned16(s_packed)) return fail(NVFP4_ERR_MISALIGNED, "s_packed must be 16-byte aligned");
-    const long long lines = (long long)((rows + 127) / 128) * (K / 64) * 32;
-    const int threads = 256;
-    const long long blocks = (lines + threads - 1) / threads;
-    if (blocks > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "scale matrix too large");
-    nvfp4::pack::pack_scales_kernel<<<(unsigned)blocks, threads, 0,
-                                      static_cast<cudaStream_t>(stream)>>>(
-        s_plain, s_packed, rows, K / 16, K / 64, lines);
+    if (!aligned16(s_plain) || !aligned16(s_packed))
+        return fail(NVFP4_ERR_MISALIGNED, "s_plain and s_packed must be 16-byte aligned");
+    const int ksteps = K / 64;
+    const dim3 grid((unsigned)((rows + 127) / 128),
+                    (unsigned)((ksteps + nvfp4::pack::KCHUNK - 1) / nvfp4::pack::KCHUNK));
+    if (grid.y > 65535) return fail(NVFP4_ERR_INVALID_ARG, "K too large for packing");
+    nvfp4::pack::pack_scales_kernel<<<grid, nvfp4::pack::ROWS, 0, static_cast<cudaStream_t>(stream)>>>(
+        s_plain, s_packed, rows, K / 16, ksteps);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launching pack_scales_kernel");
     return ok();

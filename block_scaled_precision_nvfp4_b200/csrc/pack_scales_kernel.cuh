@@ -14,32 +14,38 @@
 namespace nvfp4 {
 namespace pack {
 
-// One thread per 16-byte atom line (i, rb, ks): four 4-byte row slices in,
-// 16 bytes out.  Consecutive threads write consecutive lines.
-__global__ void pack_scales_kernel(const uint8_t* __restrict__ s, uint8_t* __restrict__ out,
-                                   int rows, int groups, int ksteps, long long lines) {
-    const long long line = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (line >= lines) return;
-    const int i = (int)(line % 32);
-    const long long atom = line / 32;
-    const int ks = (int)(atom % ksteps);
-    const long long rb = atom / ksteps;
-    uint32_t w[4];
+constexpr int ROWS = 128;  // one row block per CTA
+constexpr int KCHUNK = 8;  // K = 64 steps per CTA (32 scale bytes of each row)
+
+// CTA (rb, kc): reads the 32-byte segment of each of its 128 rows (one row
+// per thread, whole sectors), transposes through shared memory, and writes
+// the KCHUNK consecutive 512-byte atoms [rb][8*kc .. 8*kc+7] as one contiguous
+// 4 KB run.
+__global__ void __launch_bounds__(ROWS)
+pack_scales_kernel(const uint8_t* __restrict__ s, uint8_t* __restrict__ out, int rows,
+                   int groups, int ksteps) {
+    __shared__ uint32_t tile[ROWS][KCHUNK + 1];  // +1 word: conflict-free column reads
+    const int rb = blockIdx.x, kc = blockIdx.y, t = threadIdx.x;
+    const int r = rb * ROWS + t;
+    const int ks0 = kc * KCHUNK;
+    const int nks = min(KCHUNK, ksteps - ks0);
+    const uint8_t* src = s + (long long)r * groups + 4 * ks0;
+    if (r < rows && (groups % 16) == 0 && nks == KCHUNK) {
+        const uint4 a = *reinterpret_cast<const uint4*>(src);
+        const uint4 b = *reinterpret_cast<const uint4*>(src + 16);
+        tile[t][0] = a.x; tile[t][1] = a.y; tile[t][2] = a.z; tile[t][3] = a.w;
+        tile[t][4] = b.x; tile[t][5] = b.y; tile[t][6] = b.z; tile[t][7] = b.w;
+    } else {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const long long r = rb * 128 + 32 * j + i;
-        uint32_t v = 0u;
-        if (r < rows) {
-            const uint8_t* p = s + r * (long long)groups + 4 * ks;
-            if ((reinterpret_cast<uintptr_t>(p) & 3u) == 0)
-                v = *reinterpret_cast<const uint32_t*>(p);
-            else
-                v = (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) |
-                    ((uint32_t)p[3] << 24);
-        }
-        w[j] = v;
+        for (int w = 0; w < KCHUNK; ++w)
+            tile[t][w] = (r < rows && w < nks) ? *reinterpret_cast<const uint32_t*>(src + 4 * w) : 0u;
     }
-    reinterpret_cast<uint4*>(out)[line] = make_uint4(w[0], w[1], w[2], w[3]);
+    __syncthreads();
+    uint4* dst = reinterpret_cast<uint4*>(out + ((long long)rb * ksteps + ks0) * 512);
+    for (int line = t; line < nks * 32; line += ROWS) {
+        const int ksl = line >> 5, i = line & 31;
+        dst[line] = make_uint4(tile[i][ksl], tile[i + 32][ksl], tile[i + 64][ksl], tile[i + 96][ksl]);
+    }
 }
 
 }  // namespace pack

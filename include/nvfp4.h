@@ -140,8 +140,9 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, floa
 NVFP4_API size_t nvfp4_scale_layout_bytes(int rows, int K);
 
 /* Rearranges plain E4M3 group scales s_plain [rows][K/16] (device, row-major)
- * into the block-scaled MMA's scale layout in s_packed (device, 16-byte
- * aligned, nvfp4_scale_layout_bytes(rows, K) bytes, caller-owned):
+ * (16-byte aligned) into the block-scaled MMA's scale layout in s_packed
+ * (device, 16-byte aligned, nvfp4_scale_layout_bytes(rows, K) bytes,
+ * caller-owned):
  *     s_packed[rb][ks][i][j][t] = s_plain[rb*128 + 32*j + i][4*ks + t]
  * for 128-row blocks rb, K = 64 steps ks, i < 32, j < 4, t < 4 (rows past
  * `rows` are zero).  One 512-byte [i][j][t] atom is exactly what one
