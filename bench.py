@@ -244,7 +244,7 @@ KERNEL_SOURCES = {
     "w4a4": ["w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
     "via_fp8": ["via_fp8_kernel.cuh", "ptx.cuh"],
     "w4a16": ["w4a16_kernel.cuh"],
-    "grouped": ["grouped_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
+    "grouped": ["grouped_pair_kernel.cuh", "w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
 }
 
 
@@ -319,9 +319,24 @@ def run_ours(args):
         def step():
             nv.gemm_w4a16(a16, dv[1], dv[2], wl_.W.g, out=Y, stream=stream)
     elif path == "grouped":
+        # weight scales packed once per expert (model load); each step packs the routed
+        # tokens' scales per expert and runs the grouped product on pairs of SMs
         gw_list = [float(x) for x in gW]
         offs = [int(x) for x in wl_.offsets]
-        def step():
+        E = len(gw_list)
+        sw_packed = nv.nvfp4_pack_scales_grouped(dv[3].view(E * N, K // 16),
+                                                 [e * N for e in range(E + 1)], K, stream=stream)
+        sa_packed = torch.empty(nv.nvfp4_grouped_scale_layout_bytes(offs, K), dtype=torch.uint8,
+                                device=dev)
+
+        def step(mid=None):
+            nv.nvfp4_pack_scales_grouped(dv[1], offs, K, out=sa_packed, stream=stream)
+            if mid is not None:
+                mid.record(stream)
+            nv.gemm_nvfp4_w4a4_grouped_packed(dv[0], sa_packed, wl_.A.g, dv[2], sw_packed,
+                                              gw_list, offs, out=Y, stream=stream)
+
+        def plain_step():
             nv.gemm_nvfp4_w4a4_grouped(dv[0], dv[1], wl_.A.g, dv[2], dv[3], gw_list, offs,
                                        out=Y, stream=stream)
     elif path == "via_fp8":
@@ -340,7 +355,10 @@ def run_ours(args):
                 mid.record(stream)
             nv.gemm_nvfp4_w4a4_packed(dv[0], sa_packed, wl_.A.g, dv[2], sw_packed, wl_.W.g,
                                       out=Y, stream=stream)
-    launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2}.get(path, 1)
+
+        def plain_step():
+            nv.gemm_nvfp4_w4a4(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
+    launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2, "grouped": 2}.get(path, 1)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -353,7 +371,8 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] if path == "w4a4" else None
+    mids = ([torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+            if path in ("w4a4", "grouped") else None)
     with ClockSampler(dev.index) as clk:
         for i in range(args.steps):
             flush.zero_()
@@ -422,7 +441,7 @@ def run_ours(args):
         for _ in range(10):
             flush.zero_()
             p0.record(stream)
-            nv.gemm_nvfp4_w4a4(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
+            plain_step()
             p1.record(stream)
             torch.cuda.synchronize(dev)
             plain.append(p0.elapsed_time(p1))
@@ -431,7 +450,7 @@ def run_ours(args):
                  "plain_scale_entry_ms": statistics.median(plain),
                  "plain_scale_entry_tflops": flops / (statistics.median(plain) * 1e-3) / 1e12}
     kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel",
-                   "w4a16": "w4a16_kernel", "grouped": "grouped_kernel"}[path]
+                   "w4a16": "w4a16_kernel", "grouped": "grouped_pair_kernel"}[path]
     if spec["bound"] == "tensor":
         fp4_peak = bf16_peak * FP4_PER_BF16
         achieved = flops / kern_s / 1e12

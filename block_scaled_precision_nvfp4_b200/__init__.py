@@ -27,7 +27,8 @@ __all__ = [
     "nvfp4_exec_name", "nvfp4_set_fp4_kernel_disabled", "nvfp4_version",
     "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_w4a16",
     "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
-    "gemm_nvfp4_w4a4_packed", "C_FUNCTIONS",
+    "gemm_nvfp4_w4a4_packed", "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
+    "gemm_nvfp4_w4a4_grouped_packed", "C_FUNCTIONS",
 ]
 
 
@@ -88,6 +89,9 @@ C_FUNCTIONS = {
     "gemm_nvfp4_w4a4_packed": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_w4a16": (_I, [_P, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_nvfp4_w4a4_grouped": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
+    "nvfp4_grouped_scale_layout_bytes": (_Z, [_P, _I, _I]),
+    "nvfp4_pack_scales_grouped": (_I, [_P, _P, _I, _I, _P, _P]),
+    "gemm_nvfp4_w4a4_grouped_packed": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
 }
 
 _lock = threading.Lock()
@@ -293,4 +297,68 @@ def gemm_nvfp4_w4a4_grouped(A, sA, gA, W, sW, gW, offsets, out=None, stream=None
                                                 ctypes.cast(gws, ctypes.c_void_p),
                                                 ctypes.cast(off, ctypes.c_void_p), E, py, N, K,
                                                 _stream_ptr(stream)))
+    return out
+
+
+def _offsets_arg(offsets, E=None):
+    vals = [int(x) for x in offsets]
+    if E is not None and len(vals) != E + 1:
+        raise ValueError(f"offsets must hold E+1 = {E + 1} row offsets")
+    return (ctypes.c_int32 * len(vals))(*vals), len(vals) - 1
+
+
+def nvfp4_grouped_scale_layout_bytes(offsets, K: int) -> int:
+    off, E = _offsets_arg(offsets)
+    return int(load_library().nvfp4_grouped_scale_layout_bytes(ctypes.cast(off, ctypes.c_void_p),
+                                                                E, int(K)))
+
+
+def nvfp4_pack_scales_grouped(s, offsets, K=None, out=None, stream=None):
+    """Plain scales uint8 [offsets[-1], K/16] -> the grouped packed layout (each
+    group of rows starting on a 128-row block), uint8 1-D."""
+    torch = _torch()
+    rows, groups = s.shape
+    K = 16 * groups if K is None else int(K)
+    off, E = _offsets_arg(offsets)
+    if int(offsets[-1]) != rows:
+        raise ValueError("offsets must end at s.shape[0]")
+    ps = _dev_tensor(s, torch.uint8, (rows, K // 16), "s")
+    n = nvfp4_grouped_scale_layout_bytes(offsets, K)
+    if out is None:
+        out = torch.empty(max(n, 16), dtype=torch.uint8, device=s.device)
+    if out.dtype != torch.uint8 or not out.is_cuda or out.numel() < n or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous CUDA uint8 tensor of >= {n} bytes")
+    _err(load_library().nvfp4_pack_scales_grouped(ps, ctypes.cast(off, ctypes.c_void_p), E, K,
+                                                  out.data_ptr(), _stream_ptr(stream)))
+    return out
+
+
+def gemm_nvfp4_w4a4_grouped_packed(A, sA_packed, gA, W, sW_packed, gW, offsets, out=None,
+                                   stream=None):
+    """Grouped W4A4 with packed scales: sA_packed from nvfp4_pack_scales_grouped(sA,
+    offsets), sW_packed from nvfp4_pack_scales_grouped(sW.view(E*N, -1), [0, N, .., E*N])."""
+    torch = _torch()
+    M, half_k = A.shape
+    K = 2 * half_k
+    E, N = W.shape[0], W.shape[1]
+    if len(offsets) != E + 1 or int(offsets[-1]) != M:
+        raise ValueError("offsets must hold E+1 row offsets ending at A.shape[0]")
+    pa = _dev_tensor(A, torch.uint8, (M, K // 2), "A")
+    pw = _dev_tensor(W, torch.uint8, (E, N, K // 2), "W")
+    needs = (("sA_packed", sA_packed, nvfp4_grouped_scale_layout_bytes(offsets, K)),
+             ("sW_packed", sW_packed,
+              nvfp4_grouped_scale_layout_bytes([e * N for e in range(E + 1)], K)))
+    for name, t, need in needs:
+        if (not isinstance(t, torch.Tensor) or t.dtype != torch.uint8 or not t.is_cuda
+                or not t.is_contiguous() or t.numel() < need):
+            raise ValueError(f"{name} must be a contiguous CUDA uint8 tensor of >= {need} bytes")
+    off, _ = _offsets_arg(offsets, E)
+    gws = (ctypes.c_float * E)(*[float(x) for x in gW])
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
+    _err(load_library().gemm_nvfp4_w4a4_grouped_packed(
+        pa, sA_packed.data_ptr(), float(gA), pw, sW_packed.data_ptr(),
+        ctypes.cast(gws, ctypes.c_void_p), ctypes.cast(off, ctypes.c_void_p), E, py, N, K,
+        _stream_ptr(stream)))
     return out

@@ -22,6 +22,7 @@
 #include "w4a16_kernel.cuh"
 #include "via_fp8_kernel.cuh"
 #include "grouped_kernel.cuh"
+#include "grouped_pair_kernel.cuh"
 
 namespace {
 
@@ -181,6 +182,28 @@ nvfp4_status make_map_packed_sf(CUtensorMap* map, const void* base, uint64_t blo
     return NVFP4_OK;
 }
 
+// Output map of the pair kernels' TMA-store epilogue: Y bf16 [rows][N], box
+// 64 columns (128 bytes) x 32 rows, 128-byte swizzle.  Needs N % 8 == 0 (the
+// row pitch must be a multiple of 16 bytes); otherwise `valid` is 0 and the
+// kernels use plain stores (the map is then zero and never read).
+nvfp4_status make_map_out(CUtensorMap* map, const void* Y, uint64_t rows, uint64_t N, int& valid) {
+    memset(map, 0, sizeof(*map));
+    valid = 0;
+    if (N % 8 != 0) return NVFP4_OK;
+    if (!get_encoder()) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {N, rows};
+    cuuint64_t strides[1] = {N * 2};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Y), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    valid = 1;
+    return NVFP4_OK;
+}
+
 // ---------------------------------------------------------------- argument checks
 nvfp4_status check_w4a4_args(const void* A, const void* sA, const void* W, const void* sW,
                              const void* Y, int M, int N, int K) {
@@ -192,6 +215,26 @@ nvfp4_status check_w4a4_args(const void* A, const void* sA, const void* W, const
     if (!aligned16(A) || !aligned16(sA) || !aligned16(W) || !aligned16(sW) || !aligned16(Y))
         return fail(NVFP4_ERR_MISALIGNED, "every buffer must be 16-byte aligned");
     return NVFP4_OK;
+}
+
+// offsets (int32 [E+1], host): offsets[0] == 0, non-decreasing; total rows in M.
+nvfp4_status check_offsets(const int32_t* offsets_host, int E, int max_groups, int& M) {
+    if (E < 1 || E > max_groups)
+        return fail(NVFP4_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", max_groups, E);
+    if (!offsets_host) return fail(NVFP4_ERR_INVALID_ARG, "null offsets");
+    if (offsets_host[0] != 0) return fail(NVFP4_ERR_INVALID_ARG, "offsets[0] must be 0");
+    for (int e = 0; e < E; ++e)
+        if (offsets_host[e + 1] < offsets_host[e])
+            return fail(NVFP4_ERR_INVALID_ARG, "offsets must be non-decreasing");
+    M = offsets_host[E];
+    return NVFP4_OK;
+}
+
+// sum over groups of ceil(rows/128): the grouped packed layout's block count
+int64_t grouped_blocks(const int32_t* offsets_host, int E) {
+    int64_t b = 0;
+    for (int e = 0; e < E; ++e) b += (offsets_host[e + 1] - offsets_host[e] + 127) / 128;
+    return b;
 }
 
 template <typename Kern>
@@ -371,6 +414,9 @@ nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, 
         return st;
     if ((st = make_map_packed_sf(&tmSB, sW_packed, (uint64_t)(N + 127) / 128, ks, wp::NRB)) != NVFP4_OK)
         return st;
+    CUtensorMap tmY;
+    int tma_out = 0;
+    if ((st = make_map_out(&tmY, Y, (uint64_t)M, (uint64_t)N, tma_out)) != NVFP4_OK) return st;
     if ((st = set_smem(wp::w4a4_pair_kernel, wp::SMEM_BYTES, info, "w4a4_pair_kernel")) != NVFP4_OK)
         return st;
     const int tiles = ((M + wp::TILE_M - 1) / wp::TILE_M) * ((N + wp::BN - 1) / wp::BN);
@@ -387,8 +433,9 @@ nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, wp::w4a4_pair_kernel, tmA, tmB, tmSA, tmSB,
-                                       reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, wp::w4a4_pair_kernel, tmA, tmB, tmSA, tmSB, tmY,
+                                       tma_out, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K,
+                                       gA * gW);
     if (e != cudaSuccess) return cuda_fail(e, "launching w4a4_pair_kernel");
     return ok();
 }
@@ -543,6 +590,121 @@ nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t* A, const uint8_t* sA, float 
         tmA, tmW256, tmW128, tmSA, tmSW256, tmSW128, prm, reinterpret_cast<__nv_bfloat16*>(Y));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launching grouped_kernel");
+    return ok();
+}
+
+// ------------------------------------------------------------------------- grouped, packed scales
+size_t nvfp4_grouped_scale_layout_bytes(const int32_t* offsets_host, int E, int K) {
+    if (K < 64 || K % 64 != 0 || !offsets_host || E < 1 || E > nvfp4::pack::MAX_GROUPS) return 0;
+    if (offsets_host[0] != 0) return 0;
+    for (int e = 0; e < E; ++e)
+        if (offsets_host[e + 1] < offsets_host[e]) return 0;
+    return (size_t)grouped_blocks(offsets_host, E) * 128 * (size_t)(K / 16);
+}
+
+nvfp4_status nvfp4_pack_scales_grouped(const uint8_t* s_plain, const int32_t* offsets_host, int E,
+                                       int K, uint8_t* s_packed, void* stream) {
+    namespace pk = nvfp4::pack;
+    int M = 0;
+    nvfp4_status st = check_offsets(offsets_host, E, pk::MAX_GROUPS, M);
+    if (st != NVFP4_OK) return st;
+    if (K < 64 || K % 64 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "packing needs K %% 64 == 0 (got %d)", K);
+    if (M == 0) return ok();
+    if (!s_plain || !s_packed) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(s_plain) || !aligned16(s_packed))
+        return fail(NVFP4_ERR_MISALIGNED, "s_plain and s_packed must be 16-byte aligned");
+    pk::GroupedPack gp;
+    memset(&gp, 0, sizeof(gp));
+    gp.groups_n = E;
+    int64_t blocks = 0;
+    for (int e = 0; e <= E; ++e) {
+        gp.row_start[e] = offsets_host[e];
+        gp.block_start[e] = (int)blocks;
+        if (e < E) blocks += (offsets_host[e + 1] - offsets_host[e] + 127) / 128;
+    }
+    const int ksteps = K / 64;
+    const dim3 grid((unsigned)blocks, (unsigned)((ksteps + pk::KCHUNK - 1) / pk::KCHUNK));
+    if (grid.y > 65535) return fail(NVFP4_ERR_INVALID_ARG, "K too large for packing");
+    pk::pack_scales_grouped_kernel<<<grid, pk::ROWS, 0, static_cast<cudaStream_t>(stream)>>>(
+        s_plain, s_packed, gp, K / 16, ksteps);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launching pack_scales_grouped_kernel");
+    return ok();
+}
+
+nvfp4_status gemm_nvfp4_w4a4_grouped_packed(const uint8_t* A, const uint8_t* sA_packed, float gA,
+                                            const uint8_t* W, const uint8_t* sW_packed,
+                                            const float* gW_host, const int32_t* offsets_host,
+                                            int E, void* Y, int N, int K, void* stream) {
+    namespace gp = nvfp4::grouped_pair;
+    int M = 0;
+    nvfp4_status st = check_offsets(offsets_host, E, gp::MAX_EXPERTS, M);
+    if (st != NVFP4_OK) return st;
+    if (!gW_host) return fail(NVFP4_ERR_INVALID_ARG, "null gW");
+    if ((st = check_w4a4_args(A, sA_packed, W, sW_packed, Y, M, N, K)) != NVFP4_OK) return st;
+    if (K % gp::BK != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "the grouped path needs K %% 256 == 0 (got %d)", K);
+    if ((int64_t)E * N > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "E*N too large");
+    int dev;
+    DevInfo info;
+    if ((st = check_fp4_path(dev, info)) != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return ok();
+    if (info.num_sms < 2) return fail(NVFP4_ERR_CUDA, "the pair kernel needs at least two SMs");
+
+    gp::Params prm;
+    memset(&prm, 0, sizeof(prm));
+    prm.E = E;
+    prm.N = N;
+    prm.K = K;
+    int64_t total = 0, blocks = 0;
+    for (int e = 0; e < E; ++e) {
+        const int Me = offsets_host[e + 1] - offsets_host[e];
+        prm.tile_start[e] = (int)total;
+        prm.row_start[e] = offsets_host[e];
+        prm.block_start[e] = (int)blocks;
+        prm.alpha[e] = gA * gW_host[e];
+        total += gp::tiles_of_expert(Me, N);
+        blocks += (Me + 127) / 128;
+    }
+    if (total > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "too many tiles");
+    prm.tile_start[E] = (int)total;
+    prm.row_start[E] = M;
+    prm.block_start[E] = (int)blocks;
+
+    CUtensorMap tmA, tmA64, tmW, tmSA, tmSW2, tmSW1;
+    const uint64_t ks = (uint64_t)K / 64;
+    const uint64_t wblocks = (uint64_t)E * ((N + 127) / 128);
+    if ((st = make_map_u8(&tmA, A, (uint64_t)K / 2, (uint64_t)M, gp::BKB, gp::BM)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmA64, A, (uint64_t)K / 2, (uint64_t)M, gp::BKB, gp::SWAP_HALF)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_u8(&tmW, W, (uint64_t)K / 2, (uint64_t)E * N, gp::BKB, gp::BNH)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_packed_sf(&tmSA, sA_packed, (uint64_t)blocks, ks, 1)) != NVFP4_OK) return st;
+    if ((st = make_map_packed_sf(&tmSW2, sW_packed, wblocks, ks, gp::NRB)) != NVFP4_OK) return st;
+    if ((st = make_map_packed_sf(&tmSW1, sW_packed, wblocks, ks, 1)) != NVFP4_OK) return st;
+    CUtensorMap tmY;
+    int tma_out = 0;
+    if ((st = make_map_out(&tmY, Y, (uint64_t)M, (uint64_t)N, tma_out)) != NVFP4_OK) return st;
+    if ((st = set_smem(gp::grouped_pair_kernel, gp::SMEM_BYTES, info, "grouped_pair_kernel")) != NVFP4_OK)
+        return st;
+    const int pairs = total < info.num_sms / 2 ? (int)total : info.num_sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(gp::NUM_THREADS);
+    cfg.dynamicSmemBytes = gp::SMEM_BYTES;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gp::grouped_pair_kernel, tmA, tmA64, tmW, tmSA, tmSW2,
+                                       tmSW1, tmY, tma_out, prm,
+                                       reinterpret_cast<__nv_bfloat16*>(Y));
+    if (e != cudaSuccess) return cuda_fail(e, "launching grouped_pair_kernel");
     return ok();
 }
 

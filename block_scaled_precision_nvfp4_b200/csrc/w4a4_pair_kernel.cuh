@@ -12,7 +12,11 @@
 //     (tcgen05.cp.cta_group::2: one instruction serves both SMs) and issues
 //     tcgen05.mma.cta_group::2 kind::mxf4nvf4 M=256 N=256 K=64; its commits
 //     free the stage in both CTAs;
-//   * each CTA's epilogue reads its own 128 x 256 accumulator.
+//   * each CTA's epilogue reads its own 128 x 256 accumulator, releases it,
+//     and writes the BF16 tile through shared memory with TMA bulk stores
+//     (one 32-row x 128-byte box per store): a plain store from each thread's
+//     accumulator row would touch 32 rows per instruction, and those scattered
+//     stores compete with the tensor core for the shared-memory data path.
 // Against one SM per 128 x 256 tile, every SM reads half as many W bytes per
 // flop and the pair issues half as many scale copies per flop; with the
 // scales packed ahead there is no shared-memory rewrite or cross-CTA hand-off
@@ -53,6 +57,7 @@ struct Smem {
     alignas(1024) uint8_t b[STAGES][BNH * BKB];
     alignas(128) uint32_t sfa[STAGES][KSTEPS * 128];        // [ks][512-byte atom]
     alignas(128) uint32_t sfb[STAGES][NRB * KSTEPS * 128];  // [rb][ks][512-byte atom]
+    alignas(1024) uint8_t out[NUM_EPI_WARPS][32 * 128];     // each epilogue warp's staging box
     uint64_t full[STAGES];   // leader: every byte of the stage, both CTAs
     uint64_t empty[STAGES];  // each CTA: stage free (commit from the leader)
     uint64_t acc_full;       // each CTA: accumulator ready (commit from the leader)
@@ -70,6 +75,55 @@ static_assert(BN + STAGES * (SFA_COLS + SFB_COLS) <= TMEM_COLS, "TMEM budget exc
 constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
 __host__ __device__ constexpr uint32_t sfa_col(int s) { return BN + s * (SFA_COLS + SFB_COLS); }
 __host__ __device__ constexpr uint32_t sfb_col(int s) { return sfa_col(s) + SFA_COLS; }
+
+constexpr int SLAB_COLS = 64;  // columns of one output store box (128 bytes)
+
+// One epilogue warp's 32 rows (lane = row) x 128 columns, held as packed BF16
+// pairs, stored through the warp's 4 KB staging buffer as two 32 x 64 boxes.
+// The buffer holds the 128-byte swizzle of the box (16-byte chunk c of row r
+// at chunk c ^ (r & 7)), which makes the warp's shared-memory writes
+// conflict-free.  With `tma` (a valid output map, and all 32 rows of the slab
+// belonging to this output) each box leaves by one TMA bulk store, clipped at
+// N and at the map's last row; otherwise the warp copies the first `nrows`
+// rows of the box out with plain stores (rows of the slab past `nrows`, and
+// columns past N, are not written).
+__device__ __forceinline__ void store_slab(const CUtensorMap* tmY, bool tma, uint8_t* stage,
+                                           const uint32_t (&packed)[64], int row0, int nrows,
+                                           int col0, int N, __nv_bfloat16* __restrict__ Y) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (lane == 0) bulk_wait_read_all();  // the previous box has left the buffer
+        __syncwarp();
+        uint8_t* rowp = stage + lane * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int w = h * 32 + c * 4;
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(packed[w], packed[w + 1], packed[w + 2], packed[w + 3]);
+        }
+        const int x = col0 + h * SLAB_COLS;
+        if (tma) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && x < N) {
+                tma_store_2d(tmY, stage, x, row0);
+                bulk_commit_group();
+            }
+        } else {
+            __syncwarp();
+            uint16_t* y16 = reinterpret_cast<uint16_t*>(Y);
+            for (int r = 0; r < nrows; ++r) {
+                const uint8_t* src = stage + r * 128;
+                for (int c = lane; c < SLAB_COLS; c += 32)
+                    if (x + c < N)
+                        y16[(size_t)(row0 + r) * N + x + c] = *reinterpret_cast<const uint16_t*>(
+                            src + ((((c >> 3) ^ (r & 7))) << 4) + (c & 7) * 2);
+            }
+            __syncwarp();  // the box is read before the next one overwrites it
+        }
+    }
+}
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
     const int per_group = GROUP_M * num_n;
@@ -96,6 +150,8 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
                  const __grid_constant__ CUtensorMap tmB,   // W codes, box 128 B x 128 rows
                  const __grid_constant__ CUtensorMap tmSA,  // packed sA: [rb][ks*4][128 B], box (128, 16, 1)
                  const __grid_constant__ CUtensorMap tmSB,  // packed sW: same view, box (128, 16, 2)
+                 const __grid_constant__ CUtensorMap tmY,   // Y bf16 [M][N], box 64 x 32, 128B swizzle
+                 int tma_out,                               // tmY is valid (N % 8 == 0)
                  __nv_bfloat16* __restrict__ Y, int M, int N, int K, float alpha) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -224,7 +280,8 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3, half = (warp - FIRST_EPI_WARP) >> 2;
         constexpr int COLS = BN / 2, CHUNKS = COLS / 32;
-        const bool vec_ok = (N % 8) == 0;
+        static_assert(COLS == 128, "one epilogue warp stores 128 columns");
+        uint8_t* stage = sm.out[warp - FIRST_EPI_WARP];
         int tc = 0;
         for (int tile = cid; tile < tiles; tile += nclusters, ++tc) {
             int mb, nb;
@@ -248,24 +305,12 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(&sm.acc_empty, 0);
 
-            const int row = mb * TILE_M + (int)rank * BM + 32 * q + lane;
+            const int row0 = mb * TILE_M + (int)rank * BM + 32 * q;
             const int col0 = nb * BN + half * COLS;
-            if (row < M) {
-                __nv_bfloat16* yrow = Y + (size_t)row * N;
-                if (vec_ok && col0 + COLS <= N) {
-                    uint4* dst = reinterpret_cast<uint4*>(yrow + col0);
-#pragma unroll
-                    for (int j = 0; j < COLS / 8; ++j)
-                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
-                                            packed[4 * j + 3]);
-                } else {
-                    uint16_t* y16 = reinterpret_cast<uint16_t*>(yrow);
-#pragma unroll
-                    for (int j = 0; j < COLS; ++j)
-                        if (col0 + j < N) y16[col0 + j] = (uint16_t)(packed[j >> 1] >> (16 * (j & 1)));
-                }
-            }
+            if (row0 < M)
+                store_slab(&tmY, tma_out != 0, stage, packed, row0, min(32, M - row0), col0, N, Y);
         }
+        if (lane == 0) bulk_wait_all();  // staging buffers stay alive until the stores are done
     }
 
     // No CTA of the pair leaves (or frees TMEM) while the other may still use it.

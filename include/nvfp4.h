@@ -190,11 +190,42 @@ NVFP4_API nvfp4_status gemm_w4a16(const void* A_bf16, const uint8_t* W, const ui
  * `offsets_host` (int32 [E+1], host memory, offsets[0] == 0, non-decreasing)
  * is read during the call only.  Experts with fewer than 128 rows run with
  * the operands swapped (Y_e^T = W_e . A_e^T: weight rows on the MMA's M side,
- * tokens on its N side).  1 <= E <= 1024. */
+ * tokens on its N side).  1 <= E <= 256; K % 256 == 0. */
 NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t* A, const uint8_t* sA, float gA,
                                      const uint8_t* W, const uint8_t* sW,
                                      const float* gW_host, const int32_t* offsets_host,
                                      int E, void* Y_bf16, int N, int K, void* stream);
+
+/* Bytes of a grouped packed scale buffer: groups g = 0..E-1 own rows
+ * offsets[g] .. offsets[g+1]-1 and each starts on a 128-row block, so the size
+ * is sum_g ceil(rows_g/128) * 128 * K/16 (0 if an argument is invalid).
+ * `offsets_host` is int32 [E+1] in host memory, read during the call only. */
+NVFP4_API size_t nvfp4_grouped_scale_layout_bytes(const int32_t* offsets_host, int E, int K);
+
+/* nvfp4_pack_scales per group: group g's rows of s_plain [offsets[E]][K/16]
+ * are packed into the blocks starting at block b_g = sum_{h<g} ceil(rows_h/128)
+ * of s_packed (device, 16-byte aligned, nvfp4_grouped_scale_layout_bytes
+ * bytes, caller-owned); rows past a group's end are zero.  Activation scales
+ * of tokens grouped by expert are packed this way per product; the weight
+ * scales of E experts of N rows each are packed once with offsets
+ * {0, N, 2N, ..., E*N}.  1 <= E <= 256, K % 64 == 0; the offsets rules of
+ * gemm_nvfp4_w4a4_grouped.  Asynchronous on `stream`. */
+NVFP4_API nvfp4_status nvfp4_pack_scales_grouped(const uint8_t* s_plain, const int32_t* offsets_host,
+                                                 int E, int K, uint8_t* s_packed, void* stream);
+
+/* gemm_nvfp4_w4a4_grouped with packed scales: sA_packed packed by
+ * nvfp4_pack_scales_grouped with these offsets, sW_packed with offsets
+ * {0, N, ..., E*N}.  Runs on pairs of SMs (tcgen05 cta_group::2): 256-token
+ * blocks of an expert as M = 256, N = 256 tiles; an expert's last 1..128
+ * tokens (all of a small expert) swapped, 256 weight rows on the MMA's M side
+ * and 128 token slots on its N side.  Same operation, operands and errors as
+ * gemm_nvfp4_w4a4_grouped (K % 256 == 0). */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_packed(const uint8_t* A, const uint8_t* sA_packed,
+                                                      float gA, const uint8_t* W,
+                                                      const uint8_t* sW_packed,
+                                                      const float* gW_host,
+                                                      const int32_t* offsets_host, int E,
+                                                      void* Y_bf16, int N, int K, void* stream);
 
 /* ---- diagnostics ----------------------------------------------------------- */
 

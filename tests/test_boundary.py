@@ -115,3 +115,43 @@ def test_grouped_argument_errors_need_no_device():
     assert call([0] * 3, E=300) == nv.Status.INVALID_ARG     # too many experts
     assert call([0, 4, 8], K=96) == nv.Status.INVALID_ARG    # K % 32
     assert call([0, 4, 8], A=24) == nv.Status.MISALIGNED
+
+
+def test_grouped_packed_argument_errors_need_no_device():
+    lib = nv.load_library()
+    gws = (ctypes.c_float * 3)(1.0, 1.0, 1.0)
+    def call(offs, E=2, K=256, N=64, A=16):
+        o = (ctypes.c_int32 * len(offs))(*offs)
+        return lib.gemm_nvfp4_w4a4_grouped_packed(A, 16, 1.0, 16, 16,
+                                                  ctypes.cast(gws, ctypes.c_void_p),
+                                                  ctypes.cast(o, ctypes.c_void_p), E, 16, N, K, None)
+    assert call([0, 6, 5]) == nv.Status.INVALID_ARG          # decreasing
+    assert call([1, 6, 8]) == nv.Status.INVALID_ARG          # offsets[0] != 0
+    assert call([0, 0], E=0) == nv.Status.INVALID_ARG        # no experts
+    assert call([0] * 3, E=300) == nv.Status.INVALID_ARG     # too many experts
+    assert call([0, 4, 8], K=96) == nv.Status.INVALID_ARG    # K % 32
+    assert call([0, 4, 8], A=24) == nv.Status.MISALIGNED
+
+
+def test_grouped_scale_layout_bytes_is_per_group_blocks():
+    # every group starts on a 128-row block: sum of ceil(rows/128) blocks of 128 * K/16 bytes
+    assert nv.nvfp4_grouped_scale_layout_bytes([0, 1], 64) == 128 * 4
+    assert nv.nvfp4_grouped_scale_layout_bytes([0, 1, 1, 129, 385], 256) == (1 + 0 + 1 + 2) * 128 * 16
+    assert nv.nvfp4_grouped_scale_layout_bytes([0, 3278, 4751], 4096) == (26 + 12) * 128 * 256
+    E, N = 8, 14336
+    assert (nv.nvfp4_grouped_scale_layout_bytes([e * N for e in range(E + 1)], 4096)
+            == E * nv.nvfp4_scale_layout_bytes(N, 4096))
+    assert nv.nvfp4_grouped_scale_layout_bytes([0, 5], 96) == 0      # K % 64
+    assert nv.nvfp4_grouped_scale_layout_bytes([0, 5, 4], 64) == 0   # decreasing
+    assert nv.nvfp4_grouped_scale_layout_bytes([2, 5], 64) == 0      # offsets[0] != 0
+
+
+def test_grouped_pack_argument_errors_need_no_device():
+    lib = nv.load_library()
+    def call(offs, E, K=256, s=16):
+        o = (ctypes.c_int32 * len(offs))(*offs)
+        return lib.nvfp4_pack_scales_grouped(s, ctypes.cast(o, ctypes.c_void_p), E, K, 16, None)
+    assert call([0, 4, 2], 2) == nv.Status.INVALID_ARG
+    assert call([0, 4], 1, K=96) == nv.Status.INVALID_ARG
+    assert call([0, 4], 1, s=8) == nv.Status.MISALIGNED
+    assert call([0, 0, 0], 2) == nv.Status.OK                 # nothing to pack
