@@ -279,6 +279,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmA,      // A codes, box 128
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(lane_base + half * COLS + c * 32, r);
                     tmem_ld_wait();
+                    reg_fence(r);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
@@ -316,6 +317,7 @@ grouped_kernel(const __grid_constant__ CUtensorMap tmA,      // A codes, box 128
                     if (tok0 < tl.n_mma) {  // warp-uniform
                         tmem_ld_32x32b_x32(lane_base + tok0, r[c]);
                         tmem_ld_wait();
+                        reg_fence(r[c]);
                     }
                 }
                 tc_fence_before();

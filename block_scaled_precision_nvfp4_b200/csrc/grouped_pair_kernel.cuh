@@ -283,6 +283,7 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(lane_base + half * COLS + c * 32, r);
                     tmem_ld_wait();
+                    reg_fence(r);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
@@ -309,6 +310,7 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(lane_base + half * 64 + c * 32, r);
                     tmem_ld_wait();
+                    reg_fence(r);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,

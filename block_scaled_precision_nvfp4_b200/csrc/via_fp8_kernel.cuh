@@ -314,6 +314,7 @@ via_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         uint32_t v[32];
                         tmem_ld_32x32b_x32(ta + 32 * c, v);
                         tmem_ld_wait();
+                        reg_fence(v);
                         if (c == 1) {  // the whole partial is in registers: release it
                             tc_fence_before();
                             __syncwarp();

@@ -294,6 +294,7 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + half * COLS + c * 32, r);
                 tmem_ld_wait();
+                reg_fence(r);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
