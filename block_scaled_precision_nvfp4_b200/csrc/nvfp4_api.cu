@@ -247,6 +247,27 @@ nvfp4_status set_smem(Kern k, size_t bytes, const DevInfo& info, const char* nam
     return NVFP4_OK;
 }
 
+using W4a16Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                           const uint16_t*, const uint8_t*, __nv_bfloat16*, int, int, int, float, int);
+template <int NB>
+W4a16Kern w4a16_inst(bool sf_tma) {
+    return sf_tma ? nvfp4::w4a16::w4a16_kernel<NB, true> : nvfp4::w4a16::w4a16_kernel<NB, false>;
+}
+// the instantiation for `nb` row blocks per CTA (1..MAX_NB)
+W4a16Kern w4a16_kernel_for(int nb, bool sf_tma) {
+    static_assert(nvfp4::w4a16::MAX_NB == 8, "one instantiation per row-block count");
+    switch (nb) {
+        case 1: return w4a16_inst<1>(sf_tma);
+        case 2: return w4a16_inst<2>(sf_tma);
+        case 3: return w4a16_inst<3>(sf_tma);
+        case 4: return w4a16_inst<4>(sf_tma);
+        case 5: return w4a16_inst<5>(sf_tma);
+        case 6: return w4a16_inst<6>(sf_tma);
+        case 7: return w4a16_inst<7>(sf_tma);
+        default: return w4a16_inst<8>(sf_tma);
+    }
+}
+
 }  // namespace
 
 // =====================================================================================
@@ -495,35 +516,47 @@ nvfp4_status gemm_w4a16(const void* A, const uint8_t* W, const uint8_t* sW, floa
         return fail(NVFP4_ERR_NOPATH, "W4A16 has no BF16-widen kernel for sm_%d", info.sm_arch);
     if (M == 0 || N == 0) return ok();
 
-    const int total_spans = (K + k16::SPAN - 1) / k16::SPAN;
-    const int sps = (total_spans + k16::CLUSTER - 1) / k16::CLUSTER;
-    const size_t smem = k16::smem_bytes(sps);
-    nvfp4_status st = set_smem(k16::w4a16_kernel, smem, info, "w4a16_kernel");
-    if (st != NVFP4_OK) return st;
-    // the whole unified L1/shared array as shared memory: three CTAs per SM
-    cudaFuncSetAttribute(k16::w4a16_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    const int row_blocks = (N + 15) / 16;
-    const int clusters = (row_blocks + k16::WARPS - 1) / k16::WARPS;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(clusters * k16::CLUSTER);
-    cfg.blockDim = dim3(k16::THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = k16::CLUSTER;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    // one wave: blocks of 8 weight rows spread evenly over the SMs, at most
+    // MAX_NB per CTA (more CTAs than SMs only for very tall W)
+    const int nrb = (N + k16::ROWS - 1) / k16::ROWS;
+    int grid = nrb < info.num_sms ? nrb : info.num_sms;
+    int nb = (nrb + grid - 1) / grid;
+    if (nb > k16::MAX_NB) {
+        nb = k16::MAX_NB;
+        grid = (nrb + nb - 1) / nb;
+    }
+    // codes by TMA always (K % 32 == 0 keeps the row pitch a multiple of 16 bytes);
+    // scales by TMA when their row pitch K/16 is a multiple of 16 bytes too
+    const bool sf_tma = K % 256 == 0;
+    nvfp4_status st;
+    // boxes of all of a CTA's rows: CTAs own nb or nb - 1 blocks of 8 rows
+    CUtensorMap tmW, tmW1, tmS, tmS1;
+    memset(&tmW1, 0, sizeof(tmW1));
+    memset(&tmS, 0, sizeof(tmS));
+    memset(&tmS1, 0, sizeof(tmS1));
+    const uint32_t rows = (uint32_t)nb * k16::ROWS;
+    if ((st = make_map_u8(&tmW, W, (uint64_t)K / 2, (uint64_t)N, 128, rows)) != NVFP4_OK) return st;
+    if (nb > 1 && (st = make_map_u8(&tmW1, W, (uint64_t)K / 2, (uint64_t)N, 128, rows - k16::ROWS)) != NVFP4_OK)
+        return st;
+    if (sf_tma) {
+        if ((st = make_map_u8(&tmS, sW, (uint64_t)K / 16, (uint64_t)N, 64, rows,
+                              CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+            return st;
+        if (nb > 1 && (st = make_map_u8(&tmS1, sW, (uint64_t)K / 16, (uint64_t)N, 64, rows - k16::ROWS,
+                                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+            return st;
+    }
+    W4a16Kern kern = w4a16_kernel_for(nb, sf_tma);
+    const size_t smem = k16::smem_bytes(nb);
+    if ((st = set_smem(kern, smem, info, "w4a16_kernel")) != NVFP4_OK) return st;
     const float out_scale = 128.0f * gW;  // undoes the 2^-7 carried by the widened weights
     for (int m0 = 0; m0 < M; m0 += k16::TOK) {
         const int mc = M - m0 < k16::TOK ? M - m0 : k16::TOK;
         const uint16_t* a = static_cast<const uint16_t*>(A) + (size_t)m0 * K;
         __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y) + (size_t)m0 * N;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, k16::w4a16_kernel, a, W, sW, y, mc, N, K,
-                                           out_scale, sps);
+        kern<<<grid, k16::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+            tmW, tmW1, tmS, tmS1, a, sW, y, mc, N, K, out_scale, nrb);
+        cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "launching w4a16_kernel");
     }
     return ok();

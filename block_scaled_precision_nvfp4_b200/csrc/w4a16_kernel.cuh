@@ -4,44 +4,61 @@
 // row of the metrale_circuit `hardware::exec` module doc, bullet 1, for the
 // decode shape (a handful of tokens, HBM-bound on the weight stream).
 //
-// Design:
-//  * one warp owns 16 weight rows; a cluster of 8 CTAs splits K into 8
-//    slices (CTA rank = slice), each CTA's 8 warps cover the cluster's 8
-//    16-row blocks;
-//  * weights stream from HBM with 128-bit ld.global.nc (each lane 32 codes of
-//    one row per 128-code span, four spans in flight), never through smem;
+// Design (one wave of CTAs, one per SM, no cluster, no workspace):
+//  * the weight rows are cut into blocks of 8 (the MMA's N); CTA c takes a
+//    contiguous range of NB or fewer blocks, over the whole of K;
+//  * a producer warp streams the CTA's codes and group scales through a ring
+//    of shared-memory stages with TMA (1024 codes of K per stage: four
+//    128-byte-wide, 128-byte-swizzled boxes of all the CTA's rows, and one box
+//    of their scales), so many bytes stay in flight without registers;
+//  * 8 consumer warps split each stage's K: warp w takes the stage's w-th
+//    128-code span for every row block, so its activation fragments serve NB
+//    blocks; the activations arrive by cp.async into per-lane slots;
 //  * a code is widened with two shifts and one LOP3 per pair into BF16 bits
 //    worth e2m1 * 2^-126, then multiplied (bf16x2, exact) by the group scale
 //    pre-multiplied by 2^119, so each weight is e2m1 * s * 2^-7 exactly;
-//  * the MMA is mma.sync m16n8k16 BF16 with weight rows on M and tokens on N
-//    (two N tiles = 16 tokens); K is permuted inside each lane's 32 codes,
-//    and the activations are staged in shared memory in the same permuted
-//    order (conflict-free 64-bit reads);
-//  * the 8 K-slice partials are reduced in a fixed order through distributed
-//    shared memory (no global workspace), scaled by 2^7 * gW, rounded to BF16.
+//  * the MMA is mma.sync m16n8k16 BF16 with the 16 tokens on M and 8 weight
+//    rows on N (column n of the block holding row PERM(n), which makes the
+//    swizzled reads conflict-free); K is permuted inside each lane's 32 codes
+//    and the lane's activation fragments are built in the same order;
+//  * the warps' partial sums meet in shared memory and are added in a fixed
+//    warp order (deterministic), scaled by 2^7 * gW and rounded to BF16.
 #pragma once
 #include <cuda_bf16.h>
-#include <cooperative_groups.h>
 #include <cstdint>
+
+#include "ptx.cuh"
 
 namespace nvfp4 {
 namespace w4a16 {
 
-constexpr int TOK = 16;       // tokens per launch (two N = 8 MMA tiles)
-constexpr int SPAN = 128;     // codes per span (4 lanes x 32 codes per row)
-constexpr int WARPS = 8;      // 16-row blocks per CTA
-constexpr int CLUSTER = 8;    // K slices per cluster
-constexpr int THREADS = 32 * WARPS;
-constexpr int PF = 4;         // spans in flight per lane
+constexpr int TOK = 16;        // tokens per launch (the MMA's M)
+constexpr int SPAN = 128;      // codes per span (4 lanes x 32 codes per row)
+constexpr int CONSUMERS = 8;   // K splits of a stage (one span each)
+constexpr int THREADS = 32 * (CONSUMERS + 1);  // + one producer warp
+constexpr int ROWS = 8;        // weight rows per block (the MMA's N)
+constexpr int MAX_NB = 8;      // row blocks per CTA at most
+constexpr int STAGE_K = CONSUMERS * SPAN;      // 1024 codes of K per stage
+constexpr int NA = 2;          // activation spans per warp in shared memory (cp.async slots)
+constexpr int SLOT_U4 = 8 * 32;  // one span's activation chunks of a warp, in uint4
 
-static_assert(CLUSTER == WARPS, "each CTA of a cluster reduces one warp's row block");
-
-__host__ __device__ constexpr int act_row_bytes(int spans_per_slice) {
-    return spans_per_slice * 256 + 32;  // row stride = 32 mod 128: conflict-free reads
+// One stage: codes [4 column boxes][NB * 8 rows][128 B], then scales [NB * 8 rows][64 B].
+__host__ __device__ constexpr uint32_t stage_code_bytes(int nb) { return (uint32_t)nb * 4096u; }
+// (a multiple of 1024 bytes: each 128-byte-swizzled box starts on a 1024-byte boundary)
+__host__ __device__ constexpr uint32_t stage_bytes(int nb) { return ((uint32_t)nb * 4608u + 1023u) & ~1023u; }
+// roles recorded in the device error word when a wait expires
+constexpr int ROLE_W16_PRODUCER = 9, ROLE_W16_CONSUMER = 10;
+// as many stages as fit in about 150 KB, between 2 and 8
+__host__ __device__ constexpr int stages_for(int nb) {
+    return 150 * 1024 / (int)stage_bytes(nb) > 8 ? 8
+           : (150 * 1024 / (int)stage_bytes(nb) < 2 ? 2 : 150 * 1024 / (int)stage_bytes(nb));
 }
-__host__ __device__ constexpr size_t smem_bytes(int spans_per_slice) {
-    return (size_t)TOK * act_row_bytes(spans_per_slice) + (size_t)WARPS * 16 * TOK * 4;
+__host__ __device__ constexpr size_t a_ring_bytes() { return (size_t)CONSUMERS * NA * SLOT_U4 * 16; }
+__host__ __device__ constexpr size_t smem_bytes(int nb) {
+    return 1024 + (size_t)stages_for(nb) * stage_bytes(nb) + a_ring_bytes() + 2 * 8 * 8;
 }
+// the weight row (within its block of 8) held by MMA column n
+__host__ __device__ constexpr int perm_row(int n) { return (n >> 1) | ((n & 1) << 2); }
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     uint4 v;
@@ -50,19 +67,40 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     return v;
 }
 
+// 16-byte asynchronous copy global -> shared through L1 (a lane's four copies
+// of one 128-byte line land in it back to back, so each 32-byte sector leaves
+// L2 once); `src_bytes` = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 16, %2;"
+                 ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))), "l"(gsrc),
+                   "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
-// E4M3 scale byte (non-negative) -> BF16 bits of s * 2^119, packed twice.
+// E4M3 scale byte (0x00..0x7E) -> BF16 bits of s * 2^119, packed twice.  For a
+// normal byte (exponent field E >= 1) the BF16 exponent is E + 239 and the
+// three mantissa bits move up by four, i.e. (b << 4) + (239 << 7); the
+// subnormal bytes (and zero) take the float route.
 __device__ __forceinline__ uint32_t scale_pair(uint32_t b) {
-    const uint32_t E = (b >> 3) & 15u, M = b & 7u;
     uint32_t h;
-    if (E != 0) h = ((E + 239u) << 7) | (M << 4);
-    else h = __float_as_uint((float)M * 0x1p110f) >> 16;
-    return h | (h << 16);
+    if (b >= 8u) h = (b << 4) + (239u << 7);
+    else h = __float_as_uint((float)b * 0x1p110f) >> 16;
+    return h * 0x10001u;
 }
 
 // Eight codes of one word -> four BF16 pairs worth e2m1 * 2^-126, as
@@ -77,149 +115,219 @@ __device__ __forceinline__ void widen8(uint32_t q, uint32_t ss, uint32_t (&p)[4]
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-struct Span {
-    uint4 q0, q1;      // 32 codes of row g and of row g+8
-    uint32_t s0, s1;   // their two group-scale bytes (low byte: codes 0-15)
-};
-
+// NB: row blocks per CTA at most; SF_TMA: the group scales travel by TMA with
+// the codes (needs the scale row pitch K/16 to be a multiple of 16 bytes);
+// otherwise each lane loads its two scale bytes itself, one stage ahead.
+template <int NB, bool SF_TMA>
 __global__ void __launch_bounds__(THREADS, 1)
-w4a16_kernel(const uint16_t* __restrict__ A, const uint8_t* __restrict__ W,
-             const uint8_t* __restrict__ sW, __nv_bfloat16* __restrict__ Y, int M, int N, int K,
-             float out_scale, int spans_per_slice) {
-    namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int row_bytes = act_row_bytes(spans_per_slice);
-    uint8_t* act = smem;
-    float* part = reinterpret_cast<float*>(smem + (size_t)TOK * row_bytes);
+w4a16_kernel(const __grid_constant__ CUtensorMap tmW,   // codes [N][K/2], box 128 B x 8*NB rows, 128B swizzle
+             const __grid_constant__ CUtensorMap tmW1,  // the same with a box of 8*(NB-1) rows
+             const __grid_constant__ CUtensorMap tmS,   // scales [N][K/16], box 64 B x 8*NB rows (SF_TMA)
+             const __grid_constant__ CUtensorMap tmS1,  // the same with a box of 8*(NB-1) rows
+             const uint16_t* __restrict__ A, const uint8_t* __restrict__ sW,
+             __nv_bfloat16* __restrict__ Y, int M, int N, int K, float out_scale, int nrb) {
+    constexpr int STAGES = stages_for(NB);
+    constexpr uint32_t STAGE_BYTES = stage_bytes(NB);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* stages = smem;                                          // 1024-aligned stages
+    uint4* aring = reinterpret_cast<uint4*>(smem + (size_t)STAGES * STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(aring) + a_ring_bytes());
+    uint64_t* empty = full + 8;
+    __shared__ int abort_flag;
+    volatile int* abort = &abort_flag;
 
-    const int slice = (int)cluster.block_rank();
-    const int cluster_id = blockIdx.x / CLUSTER;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int span0 = slice * spans_per_slice;
-    const int total_spans = (K + SPAN - 1) / SPAN;
-    const int nspans = max(0, min(spans_per_slice, total_spans - span0));
+    const int G = gridDim.x;
+    const int rb0 = (int)((long long)blockIdx.x * nrb / G);
+    const int nb = (int)((long long)(blockIdx.x + 1) * nrb / G) - rb0;  // <= NB
+    const int nst = (K + STAGE_K - 1) / STAGE_K;
 
-    // ---- stage this slice's activations, permuted to the MMA's K order
-    for (int c = threadIdx.x; c < TOK * spans_per_slice * 4; c += THREADS) {
-        const int tt = c & 3, sp = (c >> 2) % spans_per_slice, n = c / (4 * spans_per_slice);
-        const int k = (span0 + sp) * SPAN + 32 * tt;
-        uint32_t a[16];
-        if (n < M && sp < nspans && k < K) {
-            const uint4* src = reinterpret_cast<const uint4*>(A + (size_t)n * K + k);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint4 v = __ldg(src + j);
-                a[4 * j] = v.x; a[4 * j + 1] = v.y; a[4 * j + 2] = v.z; a[4 * j + 3] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) a[j] = 0u;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], CONSUMERS);
         }
-        // a[] holds 32 bf16: element e is half (e & 1) of a[e >> 1]
-        auto el = [&](int e) -> uint32_t { return (a[e >> 1] >> (16 * (e & 1))) & 0xFFFFu; };
-        uint8_t* dst = act + (size_t)n * row_bytes + sp * 256 + tt * 8;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int w8 = 8 * (i >> 1) + 2 * (i & 1);
-            uint2 v;
-            v.x = el(w8) | (el(w8 + 4) << 16);
-            v.y = el(w8 + 1) | (el(w8 + 5) << 16);
-            *reinterpret_cast<uint2*>(dst + i * 32) = v;
-        }
+        abort_flag = 0;
+        fence_mbarrier_init();
     }
     __syncthreads();
 
-    // ---- stream this warp's 16 weight rows over the slice
-    const int rb = cluster_id * WARPS + warp;
-    const int r0 = rb * 16 + g, r1 = r0 + 8;
-    const size_t row_stride = (size_t)K / 2, srow_stride = (size_t)K / 16;
-    const bool ok0 = r0 < N, ok1 = r1 < N;
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-
-    auto load = [&](int sp, Span& s) {
-        const int k = (span0 + sp) * SPAN + 32 * t;
-        const bool in = sp < nspans && k < K;
-        s.q0 = make_uint4(0u, 0u, 0u, 0u);
-        s.q1 = s.q0;
-        s.s0 = s.s1 = 0u;
-        if (in && ok0) {
-            s.q0 = ldg_stream(W + r0 * row_stride + k / 2);
-            s.s0 = __ldg(reinterpret_cast<const uint16_t*>(sW + r0 * srow_stride + k / 16));
-        }
-        if (in && ok1) {
-            s.q1 = ldg_stream(W + r1 * row_stride + k / 2);
-            s.s1 = __ldg(reinterpret_cast<const uint16_t*>(sW + r1 * srow_stride + k / 16));
-        }
-    };
-
-    auto compute = [&](int sp, const Span& s) {
-        const uint32_t sa0 = scale_pair(s.s0 & 0xFFu), sb0 = scale_pair((s.s0 >> 8) & 0xFFu);
-        const uint32_t sa1 = scale_pair(s.s1 & 0xFFu), sb1 = scale_pair((s.s1 >> 8) & 0xFFu);
-        const uint32_t w0[4] = {s.q0.x, s.q0.y, s.q0.z, s.q0.w};
-        const uint32_t w1[4] = {s.q1.x, s.q1.y, s.q1.z, s.q1.w};
-        const uint8_t* arow0 = act + (size_t)g * row_bytes + sp * 256 + t * 8;
-        const uint8_t* arow1 = arow0 + (size_t)8 * row_bytes;
+    if (warp == CONSUMERS) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            // a CTA owns NB or NB - 1 row blocks: the box of the matching height
+            const CUtensorMap* mw = nb == NB ? &tmW : &tmW1;
+            const CUtensorMap* ms = nb == NB ? &tmS : &tmS1;
+            tma_prefetch_desc(mw);
+            if (SF_TMA) tma_prefetch_desc(ms);
+            const uint32_t bytes = (uint32_t)nb * ROWS * (512u + (SF_TMA ? 64u : 0u));
+            const int y = rb0 * ROWS;
+            int i = 0;
+            for (; i < nst; ++i) {
+                const int s = i % STAGES;
+                if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, abort, ROLE_W16_PRODUCER)) break;
+                uint8_t* st = stages + (size_t)s * STAGE_BYTES;
+                mbar_arrive_expect_tx(&full[s], bytes);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            uint32_t p0[4], p1[4];
-            widen8(w0[w], w < 2 ? sa0 : sb0, p0);
-            widen8(w1[w], w < 2 ? sa1 : sb1, p1);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int i = 2 * w + h;
-                const uint2 b0 = *reinterpret_cast<const uint2*>(arow0 + i * 32);
-                const uint2 b1 = *reinterpret_cast<const uint2*>(arow1 + i * 32);
-                mma_bf16(acc[0], p0[2 * h], p1[2 * h], p0[2 * h + 1], p1[2 * h + 1], b0.x, b0.y);
-                mma_bf16(acc[1], p0[2 * h], p1[2 * h], p0[2 * h + 1], p1[2 * h + 1], b1.x, b1.y);
+                for (int c = 0; c < 4; ++c)
+                    tma_load_2d(st + c * (NB * 1024), mw, &full[s], i * (STAGE_K / 2) + c * 128, y);
+                if (SF_TMA) tma_load_2d(st + stage_code_bytes(NB), ms, &full[s], i * (STAGE_K / 16), y);
+            }
+            // copies still in flight land before the CTA can leave
+            for (int j = (i > STAGES ? i - STAGES : 0); j < i; ++j) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&full[j % STAGES], (j / STAGES) & 1) &&
+                       globaltimer_ns() - t0 < kWaitLimitNs) {
+                }
             }
         }
+        return;  // the producer takes no part in the epilogue
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int w = warp, g = lane >> 2, t = lane & 3;
+    const int prow = perm_row(g);  // this lane's weight row within a block
+    uint4* aslot = aring + (size_t)w * NA * SLOT_U4 + lane;
+
+    // cp.async of stage i's span-w activations for this lane: tokens g and g+8, its 32 codes
+    auto issue_a = [&](int i) {
+        if (i < nst) {
+            const int k0 = i * STAGE_K + w * SPAN + 32 * t;
+            uint4* dst = aslot + (i % NA) * SLOT_U4;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int tok = g + 8 * h;
+                const bool ok = k0 < K && tok < M;
+                const uint16_t* src = ok ? A + (size_t)tok * K + k0 : A;
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    cp_async16(dst + (h * 4 + m) * 32, ok ? src + 8 * m : A, ok ? 16u : 0u);
+            }
+        }
+        cp_async_commit();  // one group per stage, empty past the end
+    };
+    // lane's own scale bytes of stage i, block b (the path without scale TMA)
+    auto scale_g = [&](int i, int b) -> uint32_t {
+        const int row = (rb0 + b) * ROWS + prow;
+        const int k0 = i * STAGE_K + w * SPAN + 32 * t;
+        if (i >= nst || b >= nb || row >= N || k0 >= K) return 0u;
+        return __ldg(reinterpret_cast<const uint16_t*>(sW + (size_t)row * (K / 16) + k0 / 16));
     };
 
-    Span buf[PF];
+    float acc[NB][4];
 #pragma unroll
-    for (int p = 0; p < PF; ++p) load(p, buf[p]);
-    for (int sp = 0; sp < nspans; sp += PF) {
+    for (int b = 0; b < NB; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
+    uint32_t sc_next[NB];
+    if (!SF_TMA) {
 #pragma unroll
-        for (int p = 0; p < PF; ++p) {
-            const Span cur = buf[p];
-            load(sp + p + PF, buf[p]);
-            if (sp + p < nspans) compute(sp + p, cur);
+        for (int b = 0; b < NB; ++b) sc_next[b] = scale_g(0, b);
+    }
+#pragma unroll
+    for (int a = 0; a < NA - 1; ++a) issue_a(a);
+
+    for (int i = 0; i < nst; ++i) {
+        const int s = i % STAGES;
+        // this stage's activation fragments (K-step 2v + h, see the file comment)
+        uint32_t af[8][4];
+        cp_async_wait<NA - 2>();
+        {
+            const uint4* src = aslot + (i % NA) * SLOT_U4;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const uint4 x0 = src[v * 32], x1 = src[(4 + v) * 32];  // tokens g, g+8
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t lo0 = h ? x0.y : x0.x, hi0 = h ? x0.w : x0.z;
+                    const uint32_t lo1 = h ? x1.y : x1.x, hi1 = h ? x1.w : x1.z;
+                    af[2 * v + h][0] = prmt(lo0, hi0, 0x5410);  // codes 2h, 2h+4 of token g
+                    af[2 * v + h][1] = prmt(lo1, hi1, 0x5410);  // the same of token g+8
+                    af[2 * v + h][2] = prmt(lo0, hi0, 0x7632);  // codes 2h+1, 2h+5
+                    af[2 * v + h][3] = prmt(lo1, hi1, 0x7632);
+                }
+            }
         }
-    }
-
-    // ---- partial sums of this slice: part[warp][row][token]
-    float* pw = part + warp * 16 * TOK;
+        issue_a(i + NA - 1);
+        uint32_t sc[NB];
+        if (!SF_TMA) {
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int tok = 8 * nt + 2 * t;
-        pw[g * TOK + tok] = acc[nt][0];
-        pw[g * TOK + tok + 1] = acc[nt][1];
-        pw[(g + 8) * TOK + tok] = acc[nt][2];
-        pw[(g + 8) * TOK + tok + 1] = acc[nt][3];
-    }
-    cluster.sync();
-
-    // ---- CTA `slice` reduces row block `slice` of the cluster over all slices
-    {
-        const int row = threadIdx.x / TOK, tok = threadIdx.x % TOK;
-        const int rrb = cluster_id * WARPS + slice;
-        const int n = rrb * 16 + row;
-        float* mine = part + slice * 16 * TOK + row * TOK + tok;
-        float s = 0.f;
+            for (int b = 0; b < NB; ++b) {
+                sc[b] = sc_next[b];
+                sc_next[b] = scale_g(i + 1, b);
+            }
+        }
+        {
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&full[s], (i / STAGES) & 1, abort, ROLE_W16_CONSUMER) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            // complete already: every lane's own wait orders its reads after the copy
+            while (!mbar_try_wait(&full[s], (i / STAGES) & 1)) {
+            }
+        }
+        const uint8_t* st = stages + (size_t)s * STAGE_BYTES;
+        // all of this lane's codes and scales of the stage first, then the MMAs
+        // interleaved across the row blocks (independent accumulators back to back)
+        uint32_t wq[NB][4], ss[NB][2];
 #pragma unroll
-        for (int c = 0; c < CLUSTER; ++c) s += *cluster.map_shared_rank(mine, c);
-        if (n < N && tok < M) Y[(size_t)tok * N + n] = __float2bfloat16_rn(s * out_scale);
+        for (int b = 0; b < NB; ++b) {
+            uint4 q = make_uint4(0u, 0u, 0u, 0u);
+            uint32_t sb2 = 0u;
+            if (b < nb) {
+                q = *reinterpret_cast<const uint4*>(
+                    st + ((w >> 1) * NB * 8 + b * 8 + prow) * 128 + ((((w & 1) * 4 + t) ^ prow) << 4));
+                sb2 = SF_TMA ? (uint32_t)*reinterpret_cast<const uint16_t*>(
+                                   st + stage_code_bytes(NB) + (b * 8 + prow) * 64 + w * 8 + t * 2)
+                             : sc[b];
+            }
+            wq[b][0] = q.x; wq[b][1] = q.y; wq[b][2] = q.z; wq[b][3] = q.w;
+            ss[b][0] = scale_pair(sb2 & 0xFFu);
+            ss[b][1] = scale_pair((sb2 >> 8) & 0xFFu);
+        }
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            uint32_t p[NB][4];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) widen8(wq[b][v], ss[b][v >> 1], p[b]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t(&a)[4] = af[2 * v + h];
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+                    if (b < nb) mma_bf16(acc[b], a[0], a[1], a[2], a[3], p[b][2 * h], p[b][2 * h + 1]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // this warp has read the stage
     }
-    cluster.sync();
+    cp_async_wait<0>();
+
+    // ---- the warps' partials meet in the (now idle) activation slots: red[w][b][lane][4]
+    named_bar_sync(1, 32 * CONSUMERS);
+    float* red = reinterpret_cast<float*>(aring);
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+        if (b < nb)
+            *reinterpret_cast<float4*>(red + ((size_t)(w * NB + b) * 32 + lane) * 4) =
+                make_float4(acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
+    named_bar_sync(1, 32 * CONSUMERS);
+
+    // ---- fixed-order sum over the warps; D[tok][n] of lane l -> Y[tok][block row PERM(n)]
+    for (int idx = threadIdx.x; idx < nb * 128; idx += 32 * CONSUMERS) {
+        const int b = idx >> 7, l = (idx >> 2) & 31, e = idx & 3;
+        float sum = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < CONSUMERS; ++ww) sum += red[((size_t)(ww * NB + b) * 32 + l) * 4 + e];
+        const int tok = (l >> 2) + 8 * (e >> 1);
+        const int row = (rb0 + b) * ROWS + perm_row(2 * (l & 3) + (e & 1));
+        if (tok < M && row < N) Y[(size_t)tok * N + row] = __float2bfloat16_rn(sum * out_scale);
+    }
 }
 
 }  // namespace w4a16

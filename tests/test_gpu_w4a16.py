@@ -36,8 +36,12 @@ def test_decode_workload_full_output():
     check(bf16_to_f64(y), ref, "w4a16 decode")
 
 
-SHAPES = [(1, 8, 32), (3, 24, 96), (16, 100, 160), (16, 136, 1024), (5, 520, 4128),
-          (17, 64, 256), (40, 200, 512), (16, 2048, 14336)]
+# Rows spread over one wave of CTAs in blocks of 8: these shapes give 1 to 8
+# blocks per CTA (and more CTAs than SMs for the tallest), odd N, a single row,
+# K not a multiple of the 128-code span, and token counts around 16.
+SHAPES = [(1, 8, 32), (1, 1, 32), (2, 101, 288), (3, 24, 96), (16, 100, 160),
+          (16, 136, 1024), (5, 520, 4128), (7, 3000, 544), (17, 64, 256), (40, 200, 512),
+          (16, 2048, 14336), (16, 12000, 256)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
