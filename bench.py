@@ -72,6 +72,8 @@ WORKLOADS = {
     "w4a16": dict(path="w4a16", bound="hbm", desc="W4A16 decode 16x5376x14336"),
     "grouped": dict(path="grouped", bound="tensor", desc="grouped MoE W4A4, 8 experts"),
     "tiny": dict(path="w4a4", bound="tensor", desc="tiny W4A4 128x256x256"),
+    "quantize": dict(path="quantize", bound="hbm",
+                     desc="NVFP4 quantiser of the FFN-down activations, BF16 4096x14336"),
 }
 
 
@@ -83,6 +85,8 @@ def make_workload(name):
         return wl.w4a16_decode()
     if name == "grouped":
         return wl.grouped_w4a4()
+    if name == "quantize":
+        return wl.activations_bf16()
     return wl.ffn_down_w4a4()
 
 
@@ -91,7 +95,9 @@ def algorithmic(wl_, path):
     M, N, K = wl_.M, wl_.N, wl_.K
     flops = 2.0 * M * N * K
     ybytes = M * N * 2
-    if path == "w4a16":
+    if path == "quantize":
+        # X read once; codes, packed scales and g written (the two-pass amax reads X twice)
+        return 0.0, M * K * 2 + M * K // 2 + M * K // 16 + 4
         return flops, N * K // 2 + N * K // 16 + M * K * 2 + ybytes
     if path == "grouped":
         return flops, wl_.E * (N * K // 2 + N * K // 16) + M * (K // 2 + K // 16) + ybytes
@@ -166,6 +172,10 @@ class ClockSampler:
 def _oracle_rows(wl_, rows):
     """The FP64 oracle on the first `rows` output rows of the workload."""
     import oracle
+    if wl_.N == 0:
+        from oracle import quantize as oq
+        oq.quantize_nvfp4_bf16(wl_.A_bf16[:rows])
+        return
     if wl_.A_bf16 is not None:
         oracle.gemm_w4a16(wl_.A_bf16[:rows], wl_.W.codes, wl_.W.scales, wl_.W.g, rows, wl_.N,
                           wl_.K)
@@ -189,9 +199,12 @@ def oracle_rows_for(seconds, wl_, rate_probe_rows=2):
 
 
 def time_oracle(wl_, rows):
+    """(throughput in the workload's unit, seconds) of the oracle on `rows` rows."""
     t0 = time.perf_counter()
     _oracle_rows(wl_, rows)
     dt = time.perf_counter() - t0
+    if wl_.N == 0:  # the quantiser: GB/s of its algorithmic bytes
+        return rows * wl_.K * (2 + 0.5 + 1 / 16) / dt / 1e9, dt
     return 2.0 * rows * wl_.N * wl_.K / dt / 1e12, dt
 
 
@@ -199,9 +212,11 @@ def cpu_baseline(wl_, seconds=12.0):
     import oracle
     rows = oracle_rows_for(seconds, wl_)
     tflops, dt = time_oracle(wl_, rows)
-    return {"value": tflops, "unit": "TFLOP/s", "cores": oracle.default_threads(),
+    return {"value": tflops, "unit": "GB/s" if wl_.N == 0 else "TFLOP/s",
+            "cores": oracle.default_threads(),
             "kind": "oracle",
-            "sample": f"first {rows} of {wl_.M} rows of Y ({rows}x{wl_.N}x{wl_.K}), {dt:.1f} s"}
+            "sample": (f"first {rows} of {wl_.M} rows of X ({rows}x{wl_.K}), {dt:.1f} s" if wl_.N == 0 else
+                       f"first {rows} of {wl_.M} rows of Y ({rows}x{wl_.N}x{wl_.K}), {dt:.1f} s")}
 
 
 def run_reference(args):
@@ -245,6 +260,7 @@ KERNEL_SOURCES = {
     "via_fp8": ["via_fp8_kernel.cuh", "ptx.cuh"],
     "w4a16": ["w4a16_kernel.cuh"],
     "grouped": ["grouped_pair_kernel.cuh", "w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
+    "quantize": ["quantize_kernel.cuh"],
 }
 
 
@@ -302,7 +318,9 @@ def run_ours(args):
         return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
 
     # host copies of the inputs (pinned) and their device twins
-    if path == "w4a16":
+    if path == "quantize":
+        host = [wl_.A_bf16.view(np.int16)]
+    elif path == "w4a16":
         host = [wl_.A_bf16.view(np.int16), wl_.W.codes, wl_.W.scales]
     elif path == "grouped":
         Wc, Ws, gW = wlm.stack_experts(wl_)
@@ -314,7 +332,18 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    if path == "w4a16":
+    if path == "quantize":
+        xq = dv[0].view(torch.bfloat16)
+        q_ws = torch.empty(16, dtype=torch.uint8, device=dev)
+        # codes, scales in the product's packed layout, and g (what the product consumes)
+        Y = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        q_out = (Y, None, torch.empty(nv.nvfp4_scale_layout_bytes(M, K), dtype=torch.uint8,
+                                      device=dev), torch.empty(4, dtype=torch.float32, device=dev))
+
+        def step():
+            nv.nvfp4_quantize_bf16(xq, plain=False, packed=True, workspace=q_ws, stream=stream,
+                                   out=q_out)
+    elif path == "w4a16":
         a16 = dv[0].view(torch.bfloat16)
         def step():
             nv.gemm_w4a16(a16, dv[1], dv[2], wl_.W.g, out=Y, stream=stream)
@@ -358,7 +387,7 @@ def run_ours(args):
 
         def plain_step():
             nv.gemm_nvfp4_w4a4(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
-    launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2, "grouped": 2}.get(path, 1)
+    launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2, "grouped": 2, "quantize": 2}.get(path, 1)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -393,12 +422,14 @@ def run_ours(args):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         t_ms = float(tt.item())
     value = world * flops / (t_ms * 1e-3) / 1e12
+    if path == "quantize":  # no flops: whole-job GB/s of the algorithmic bytes
+        value = world * alg_bytes / (t_ms * 1e-3) / 1e9
 
     # end to end through the public API: pinned host inputs -> device -> call -> host result
     e2e = None
     if not args.no_e2e:
         hp = [torch.from_numpy(np.ascontiguousarray(h)).pin_memory() for h in host]
-        hY = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        hY = torch.empty(tuple(Y.shape), dtype=Y.dtype).pin_memory()
         e_steps = max(1, min(args.steps, 20))
 
         def e2e_step():
@@ -424,8 +455,10 @@ def run_ours(args):
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             te = float(tt.item())
         h2d = sum(x.numel() * x.element_size() for x in hp)
-        e2e = {"value": world * flops / (te * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hY.numel() * 2,
+        e2e = {"value": (world * alg_bytes / (te * 1e-3) / 1e9 if path == "quantize"
+                         else world * flops / (te * 1e-3) / 1e12),
+               "unit": "GB/s" if path == "quantize" else "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hY.numel() * hY.element_size(),
                "ms_per_step": te}
 
     bf16_peak, hbm_peak, peak_src = peaks()
@@ -450,7 +483,8 @@ def run_ours(args):
                  "plain_scale_entry_ms": statistics.median(plain),
                  "plain_scale_entry_tflops": flops / (statistics.median(plain) * 1e-3) / 1e12}
     kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel",
-                   "w4a16": "w4a16_kernel", "grouped": "grouped_pair_kernel"}[path]
+                   "w4a16": "w4a16_kernel", "grouped": "grouped_pair_kernel",
+                   "quantize": "quantize_bf16_kernel (+ amax_bf16_kernel)"}[path]
     if spec["bound"] == "tensor":
         fp4_peak = bf16_peak * FP4_PER_BF16
         achieved = flops / kern_s / 1e12
@@ -462,23 +496,28 @@ def run_ours(args):
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "peak_note": f"{peak_src} copy bandwidth",
                 "algorithmic_bytes": alg_bytes}
-        # context: a plain library streaming read of the same weight bytes under the
-        # same L2 flush (the 256 MiB write leaves L2 dirty, and the read's misses
-        # must write those lines back), as the practical ceiling of this regime
-        wbytes = dv[1].view(torch.int32)
+        # context: a plain library copy of the same bytes (the input of the path's main
+        # stream) under the same L2 flush, counted as read + write like the measured copy
+        # peak: the 256 MiB flush write leaves L2 dirty, and the misses of a short kernel
+        # must write those lines back, so this is the practical ceiling of the regime
+        wsrc = dv[0] if path == "quantize" else dv[1]
+        wdst = torch.empty_like(wsrc)
         r0 = torch.cuda.Event(enable_timing=True); r1 = torch.cuda.Event(enable_timing=True)
         reads = []
         for _ in range(10):
             flush.zero_()
             r0.record(stream)
-            wbytes.sum(dtype=torch.int64)
+            wdst.copy_(wsrc)
             r1.record(stream)
             torch.cuda.synchronize(dev)
             reads.append(r0.elapsed_time(r1))
         rd = statistics.median(reads)
-        extra = {"stream_read_same_flush_us": rd * 1e3,
-                 "stream_read_same_flush_gbs": dv[1].numel() / (rd * 1e-3) / 1e9,
-                 "stream_read_note": "torch int64 sum over the W codes after the same flush"}
+        nbytes = wsrc.numel() * wsrc.element_size()
+        extra = {"copy_same_bytes_same_flush_us": rd * 1e3,
+                 "copy_same_bytes_same_flush_gbs": 2 * nbytes / (rd * 1e-3) / 1e9,
+                 "copy_note": ("torch copy of the " + ("input activations" if path == "quantize"
+                                                       else "weight codes")
+                               + " after the same flush; GB/s counts read + write")}
     else:
         # each (row, column, group) update is two FP32 operations (the scale product
         # and the FMA into the accumulator) on 128 FP32 lanes per SM:
@@ -495,11 +534,13 @@ def run_ours(args):
                  "kernel_ms": kern_s * 1e3})
     roof.update(extra)
     line = {
-        "metric": METRIC if args.workload == "ffn_down" else f"{spec['desc']} TFLOP/s",
-        "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "metric": (METRIC if args.workload == "ffn_down" else
+                   f"{spec['desc']} " + ("GB/s" if path == "quantize" else "TFLOP/s")),
+        "value": value, "unit": "GB/s" if path == "quantize" else "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": ("bf16 x nvfp4(e2m1, e4m3 group scales) -> f32 accumulate -> bf16"
+        "dtype": ("bf16 -> nvfp4 (fp32 scale arithmetic)" if path == "quantize" else
+                  "bf16 x nvfp4(e2m1, e4m3 group scales) -> f32 accumulate -> bf16"
                   if path == "w4a16" else
                   "nvfp4(e2m1 x e2m1, e4m3 group scales) -> f32 accumulate -> bf16"),
         "data": "synthetic",

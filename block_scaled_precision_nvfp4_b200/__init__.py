@@ -28,7 +28,7 @@ __all__ = [
     "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_w4a16",
     "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
     "gemm_nvfp4_w4a4_packed", "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
-    "gemm_nvfp4_w4a4_grouped_packed", "C_FUNCTIONS",
+    "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "C_FUNCTIONS",
 ]
 
 
@@ -92,6 +92,8 @@ C_FUNCTIONS = {
     "nvfp4_grouped_scale_layout_bytes": (_Z, [_P, _I, _I]),
     "nvfp4_pack_scales_grouped": (_I, [_P, _P, _I, _I, _P, _P]),
     "gemm_nvfp4_w4a4_grouped_packed": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
+    "nvfp4_quantize_workspace_bytes": (_Z, []),
+    "nvfp4_quantize_bf16": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
 }
 
 _lock = threading.Lock()
@@ -232,6 +234,50 @@ def nvfp4_pack_scales(s, K=None, out=None, stream=None):
         raise ValueError(f"out must be a contiguous CUDA uint8 tensor of >= {n} bytes")
     _err(load_library().nvfp4_pack_scales(ps, rows, K, out.data_ptr(), _stream_ptr(stream)))
     return out
+
+
+def nvfp4_quantize_bf16(x, plain=True, packed=True, workspace=None, stream=None, out=None):
+    """Two-level NVFP4 quantisation of a BF16 [rows, K] CUDA tensor on the GPU.
+
+    Returns (codes uint8 [rows, K/2], scales uint8 [rows, K/16] or None,
+    packed scales uint8 1-D or None, g: a 1-element float32 CUDA tensor).
+    `out`, if given, is such a tuple of preallocated tensors to write into."""
+    torch = _torch()
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise TypeError("x must be a 2-D torch.Tensor")
+    rows, K = x.shape
+    px = _dev_tensor(x, torch.bfloat16, (rows, K), "x")
+    dev = x.device
+    if out is not None:
+        codes, scales, sp, g = out
+    else:
+        codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((rows, K // 16), dtype=torch.uint8, device=dev) if plain else None
+        sp = (torch.empty(max(nvfp4_scale_layout_bytes(rows, K), 16), dtype=torch.uint8, device=dev)
+              if packed else None)
+        g = torch.empty(4, dtype=torch.float32, device=dev)
+    _dev_tensor(codes, torch.uint8, (rows, K // 2), "codes")
+    if scales is not None:
+        _dev_tensor(scales, torch.uint8, (rows, K // 16), "scales")
+    if sp is not None:
+        need = nvfp4_scale_layout_bytes(rows, K)
+        if sp.dtype != torch.uint8 or not sp.is_cuda or not sp.is_contiguous() or sp.numel() < need:
+            raise ValueError(f"packed scales must be a contiguous CUDA uint8 tensor of >= {need} bytes")
+    if g.dtype != torch.float32 or not g.is_cuda or g.numel() < 1:
+        raise ValueError("g must be a CUDA float32 tensor")
+    lib = load_library()
+    nws = int(lib.nvfp4_quantize_workspace_bytes())
+    if workspace is None:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=dev)
+    if (not isinstance(workspace, torch.Tensor) or not workspace.is_cuda
+            or not workspace.is_contiguous() or workspace.numel() * workspace.element_size() < nws):
+        raise ValueError(f"workspace must be a contiguous CUDA tensor of >= {nws} bytes")
+    _err(lib.nvfp4_quantize_bf16(px, rows, K, codes.data_ptr(),
+                                 scales.data_ptr() if scales is not None else None,
+                                 sp.data_ptr() if sp is not None else None, g.data_ptr(),
+                                 workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
+    return codes, scales, sp, g[:1]
 
 
 def gemm_nvfp4_w4a4_packed(A, sA_packed, gA, W, sW_packed, gW, out=None, stream=None):

@@ -23,6 +23,7 @@
 #include "via_fp8_kernel.cuh"
 #include "grouped_kernel.cuh"
 #include "grouped_pair_kernel.cuh"
+#include "quantize_kernel.cuh"
 
 namespace {
 
@@ -410,6 +411,62 @@ nvfp4_status nvfp4_pack_scales(const uint8_t* s_plain, int rows, int K, uint8_t*
         s_plain, s_packed, rows, K / 16, ksteps);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launching pack_scales_kernel");
+    return ok();
+}
+
+// ------------------------------------------------------------------------- quantiser
+size_t nvfp4_quantize_workspace_bytes(void) { return NVFP4_QUANTIZE_WORKSPACE_BYTES; }
+
+nvfp4_status nvfp4_quantize_bf16(const void* X, int rows, int K, uint8_t* codes, uint8_t* scales,
+                                 uint8_t* scales_packed, float* g_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    namespace q = nvfp4::quant;
+    if (rows < 0) return fail(NVFP4_ERR_INVALID_ARG, "rows must be >= 0 (got %d)", rows);
+    if (K < 16 || K % 16 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "K must be a positive multiple of 16 (got %d)", K);
+    if (!g_out || !workspace || (rows > 0 && (!X || !codes)))
+        return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!scales && !scales_packed)
+        return fail(NVFP4_ERR_INVALID_ARG, "at least one of scales and scales_packed is needed");
+    if (scales_packed && K % 64 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "packed scales need K %% 64 == 0 (got %d)", K);
+    if (workspace_bytes < NVFP4_QUANTIZE_WORKSPACE_BYTES)
+        return fail(NVFP4_ERR_INVALID_ARG, "the workspace needs %d bytes (got %zu)",
+                    NVFP4_QUANTIZE_WORKSPACE_BYTES, workspace_bytes);
+    if ((X && !aligned16(X)) || (codes && !aligned16(codes)) || (scales && !aligned16(scales)) ||
+        (scales_packed && !aligned16(scales_packed)) || !aligned16(workspace) ||
+        reinterpret_cast<uintptr_t>(g_out) % 4 != 0)
+        return fail(NVFP4_ERR_MISALIGNED, "buffers must be 16-byte aligned (g_out 4-byte)");
+    if ((long long)rows * K > (1ll << 40)) return fail(NVFP4_ERR_INVALID_ARG, "tensor too large");
+    int dev;
+    DevInfo info;
+    if (!current_device(dev, info)) return fail(NVFP4_ERR_CUDA, "cannot query the current CUDA device");
+    if (info.sm_arch != 100)
+        return fail(NVFP4_ERR_NOPATH, "the quantiser is compiled for sm_100 only (device sm_%d)",
+                    info.sm_arch);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned* amax = static_cast<unsigned*>(workspace);
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the quantiser workspace");
+    const size_t total = (size_t)rows * K;
+    const size_t n16 = total / 8;
+    if (total > 0) {
+        size_t blocks = (n16 + q::AMAX_THREADS - 1) / q::AMAX_THREADS;
+        const size_t cap = (size_t)info.num_sms * 4;
+        if (blocks > cap) blocks = cap;
+        if (blocks == 0) blocks = 1;
+        const uint16_t* x16 = static_cast<const uint16_t*>(X);
+        q::amax_bf16_kernel<<<(unsigned)blocks, q::AMAX_THREADS, 0, st>>>(
+            reinterpret_cast<const uint4*>(X), n16, x16 + n16 * 8, (int)(total - n16 * 8), amax);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launching amax_bf16_kernel");
+    }
+    // at least one CTA, so that g_out is written for an empty tensor too
+    const dim3 grid((unsigned)(rows > 0 ? (rows + q::TILE_ROWS - 1) / q::TILE_ROWS : 1),
+                    (unsigned)((K + q::TILE_COLS - 1) / q::TILE_COLS));
+    if (grid.y > 65535) return fail(NVFP4_ERR_INVALID_ARG, "K too large (got %d)", K);
+    q::quantize_bf16_kernel<<<grid, q::THREADS, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(X), rows, K, amax, codes, scales, scales_packed, g_out);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launching quantize_bf16_kernel");
     return ok();
 }
 

@@ -1,0 +1,189 @@
+// quantize_kernel.cuh -- BF16 activations -> NVFP4 (E2M1 codes, E4M3 group
+// scales, FP32 per-tensor scale): the step ahead of the W4A4 matmul.
+//
+// Two-level recipe of the FFN-down workload ("per-16 scale = amax/6 rounded to
+// E4M3 and a per-tensor FP32 scale = tensor amax/(6*448)"), every step an IEEE
+// FP32 operation rounded to nearest even, in this order:
+//     g      = amax|X| / 2688                         (1 when amax = 0)
+//     q      = amax_b / (6 * g)                       per 16 consecutive k
+//     s_b    = E4M3(q), nearest even, satfinite       (cvt.rn.satfinite)
+//     t      = x / (s * g)                            (+-0 when s = 0)
+//     code   = sign(t) | E2M1(|t|), nearest even, satfinite
+// Two launches: a reduction of amax into a caller-owned scratch word (the
+// magnitude bits of BF16 order like the values, so the maximum is an integer
+// maximum), then the quantiser proper, one CTA per 128 rows x 256 columns,
+// which also writes the scales in the block-scaled MMA's packed layout
+// (pack_scales_kernel.cuh) so the matmul needs no separate packing pass.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace nvfp4 {
+namespace quant {
+
+constexpr int AMAX_THREADS = 512;
+constexpr int TILE_ROWS = 128;   // one packed 128-row block
+constexpr int TILE_COLS = 256;   // 16 groups: four K = 64 steps
+constexpr int THREADS = 256;     // 8 warps x 16 rows
+constexpr int QB = 4;            // row segments of a warp in flight at once
+
+// max over |x| as BF16 magnitude bits (15 bits), into *amax_bits (atomic max)
+__global__ void __launch_bounds__(AMAX_THREADS)
+amax_bf16_kernel(const uint4* __restrict__ x, size_t n16, const uint16_t* __restrict__ tail,
+                 int ntail, unsigned* amax_bits) {
+    unsigned m = 0;
+    for (size_t i = blockIdx.x * (size_t)AMAX_THREADS + threadIdx.x; i < n16;
+         i += (size_t)gridDim.x * AMAX_THREADS) {
+        const uint4 v = __ldcs(x + i);
+        const unsigned a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+        const unsigned b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+        const unsigned c = __vmaxu2(a, b);
+        m = max(m, max(c & 0xFFFFu, c >> 16));
+    }
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < ntail; i += AMAX_THREADS) m = max(m, (unsigned)(tail[i] & 0x7FFFu));
+    m = __reduce_max_sync(0xffffffffu, m);
+    __shared__ unsigned wmax[AMAX_THREADS / 32];
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        unsigned v = threadIdx.x < AMAX_THREADS / 32 ? wmax[threadIdx.x] : 0u;
+        v = __reduce_max_sync(0xffffffffu, v);
+        if (threadIdx.x == 0 && v != 0) atomicMax(amax_bits, v);
+    }
+}
+
+__device__ __forceinline__ float global_scale(unsigned amax_bits) {
+    const float amax = __uint_as_float(amax_bits << 16);
+    return amax > 0.f ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+}
+
+// q >= 0 -> E4M3 byte, nearest even, saturating at 448
+__device__ __forceinline__ uint32_t e4m3_satfinite(float q) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(q), "f"(q));
+    return r & 0xFFu;
+}
+// E4M3 byte -> its value (exact)
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(b | (b << 8))));
+    return __half2float(__ushort_as_half((uint16_t)(h2 & 0xFFFFu)));
+}
+// eight magnitudes |t0| .. |t7| -> eight E2M1 magnitude codes, packed with
+// element 2j in the low nibble of byte j (cvt puts its first operand in the high
+// nibble)
+__device__ __forceinline__ uint32_t e2m1x8_mag(const float (&t)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(fabsf(t[0])), "f"(fabsf(t[1])), "f"(fabsf(t[2])), "f"(fabsf(t[3])),
+          "f"(fabsf(t[4])), "f"(fabsf(t[5])), "f"(fabsf(t[6])), "f"(fabsf(t[7])));
+    return r;
+}
+
+// One CTA: rows [128*blockIdx.x, +128) x columns [256*blockIdx.y, +256).
+// Warp w takes rows 16w .. 16w+15; lane l holds columns 8l .. 8l+7 of the row
+// (lanes 2j and 2j+1 make group j).
+__global__ void __launch_bounds__(THREADS)
+quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
+                     const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
+                     uint8_t* __restrict__ scales, uint8_t* __restrict__ scales_packed,
+                     float* __restrict__ g_out) {
+    __shared__ uint32_t sc[TILE_ROWS][TILE_COLS / 64 + 1];  // [row][K=64 step] four scale bytes
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = blockIdx.x * TILE_ROWS, c0 = blockIdx.y * TILE_COLS;
+    const float g = global_scale(*amax_bits);
+    const float d6 = __fmul_rn(6.0f, g);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
+    const int col = c0 + 8 * lane;
+    const bool col_ok = col < K;  // K % 16 == 0: a lane's 8 columns are all in or all out
+
+    // this warp's 16 row segments, QB at a time in flight before any is used
+    constexpr int RPW = TILE_ROWS / 8;  // rows per warp
+#pragma unroll 1
+    for (int i0 = 0; i0 < RPW; i0 += QB) {
+        uint4 vin[QB];
+#pragma unroll
+        for (int i = 0; i < QB; ++i) {
+            const int row = r0 + warp * RPW + i0 + i;
+            vin[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (col_ok && row < rows) vin[i] = __ldcs(reinterpret_cast<const uint4*>(X + (size_t)row * K + col));
+        }
+#pragma unroll
+    for (int i = 0; i < QB; ++i) {
+        const int rl = warp * RPW + i0 + i;
+        const int row = r0 + rl;
+        const bool ok = col_ok && row < rows;
+        const uint4 v = vin[i];
+        // group amax over the lane pair (integer max of the magnitude bits)
+        const unsigned a = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                    __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+        unsigned m = max(a & 0xFFFFu, a >> 16);
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        const float amax_b = __uint_as_float(m << 16);
+        const uint32_t sb = e4m3_satfinite(__fdiv_rn(amax_b, d6));
+        const float den = __fmul_rn(e4m3_value(sb), g);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float t[8];
+        uint32_t sgn = 0u;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            // element e is half (e & 1) of word e >> 1
+            const uint32_t h = (e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16);
+            const float xe = __uint_as_float(h);
+            t[e] = den > 0.f ? __fdiv_rn(xe, den) : xe * 0.0f;
+            sgn |= (__float_as_uint(t[e]) >> 31) << (4 * e + 3);
+        }
+        const uint32_t out = e2m1x8_mag(t) | sgn;
+        if (ok) *reinterpret_cast<uint32_t*>(codes + (size_t)row * (K / 2) + col / 2) = out;
+        // the group's scale byte: lane 2j holds group j; gather four groups (one K = 64
+        // step) into one word in shared memory
+        const uint32_t b0 = __shfl_sync(0xffffffffu, sb, (lane & ~7) + 0);
+        const uint32_t b1 = __shfl_sync(0xffffffffu, sb, (lane & ~7) + 2);
+        const uint32_t b2 = __shfl_sync(0xffffffffu, sb, (lane & ~7) + 4);
+        const uint32_t b3 = __shfl_sync(0xffffffffu, sb, (lane & ~7) + 6);
+        const uint32_t word = row < rows ? (b0 | (b1 << 8) | (b2 << 16) | (b3 << 24)) : 0u;
+        if ((lane & 7) == 0) sc[rl][lane >> 3] = col_ok ? word : 0u;
+    }
+    }
+    __syncthreads();
+
+    const int nks = min(TILE_COLS / 64, (K - c0 + 63) / 64);  // K = 64 steps of this tile
+    if (scales) {
+        // plain [rows][K/16]: each row's 4..16 bytes of this tile
+        for (int idx = threadIdx.x; idx < TILE_ROWS * (TILE_COLS / 64); idx += THREADS) {
+            const int rl = idx >> 2, ks = idx & 3, row = r0 + rl;
+            const int g0 = c0 / 16 + 4 * ks;  // first group of the word
+            if (row < rows && g0 < K / 16) {
+                uint8_t* dst = scales + (size_t)row * (K / 16) + g0;
+                const uint32_t wv = sc[rl][ks];
+                const int n = min(4, K / 16 - g0);
+                if (n == 4 && (K / 16) % 4 == 0) {
+                    *reinterpret_cast<uint32_t*>(dst) = wv;  // 4-byte aligned
+                } else {
+                    for (int b = 0; b < n; ++b) dst[b] = (uint8_t)(wv >> (8 * b));
+                }
+            }
+        }
+    }
+    if (scales_packed && K % 64 == 0) {
+        // packed[rb][ks][i][j][t] = s[128 rb + 32 j + i][4 ks + t]: this tile's nks atoms,
+        // contiguous, one 16-byte line (i) per thread and step
+        const int ksteps = K / 64, ks0 = c0 / 64;
+        uint4* dst = reinterpret_cast<uint4*>(scales_packed + ((size_t)blockIdx.x * ksteps + ks0) * 512);
+        for (int line = threadIdx.x; line < nks * 32; line += THREADS) {
+            const int ksl = line >> 5, i = line & 31;
+            dst[line] = make_uint4(sc[i][ksl], sc[i + 32][ksl], sc[i + 64][ksl], sc[i + 96][ksl]);
+        }
+    }
+}
+
+}  // namespace quant
+}  // namespace nvfp4

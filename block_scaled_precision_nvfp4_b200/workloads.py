@@ -194,6 +194,14 @@ def w4a16_decode(M: int = 16, N: int = 5376, K: int = 14336, seed_a: int = 0,
                     notes="A bf16 N(0,1) seed %d, W~N(0,0.02) seed %d" % (seed_a, seed_w))
 
 
+def activations_bf16(M: int = 4096, K: int = 14336, seed: int = 0) -> Workload:
+    """The FFN-down activations before quantisation: BF16 N(0,1) [M,K] (seed 0)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    A = to_bf16_bits(rng.standard_normal((M, K), dtype=np.float32))
+    return Workload(f"quantize_bf16_{M}x{K}", M, 0, K, A_bf16=A,
+                    notes="X bf16 N(0,1) seed %d" % seed)
+
+
 def zipf_routing(tokens: int, E: int, s: float, seed: int) -> np.ndarray:
     """Top-1 expert per token from a multinomial with p_e proportional to (e+1)^-s."""
     p = (np.arange(1, E + 1, dtype=np.float64)) ** (-s)

@@ -152,6 +152,40 @@ NVFP4_API size_t nvfp4_scale_layout_bytes(int rows, int K);
 NVFP4_API nvfp4_status nvfp4_pack_scales(const uint8_t* s_plain, int rows, int K,
                                          uint8_t* s_packed, void* stream);
 
+/* ---- activation quantiser (the step ahead of the W4A4 product) ----------- */
+
+/* Bytes of device scratch nvfp4_quantize_bf16 needs (a constant). */
+#define NVFP4_QUANTIZE_WORKSPACE_BYTES 16
+NVFP4_API size_t nvfp4_quantize_workspace_bytes(void);
+
+/* Two-level NVFP4 quantisation of a BF16 matrix, the encoding the W4A4 product
+ * consumes (the FFN-down workload: "per-16 scale = amax/6 rounded to E4M3 and a
+ * per-tensor FP32 scale = tensor amax/(6*448)", read as two levels: the block
+ * scale relative to the per-tensor one).  Every step is an IEEE FP32 operation
+ * rounded to nearest even, in this order:
+ *     g    = amax|X| / 2688                (g = 1 when X is all zero)
+ *     s_b  = E4M3(amax_b / (6 g))          per 16 consecutive k of a row,
+ *                                          nearest even, saturating at 448
+ *     code = sign(t) | E2M1(|t|),  t = x / (s_b g)   (t = +-0 when s_b = 0),
+ *                                          nearest even, saturating at 6
+ *   X_bf16         device, [rows][K] BF16 row-major, finite values
+ *   codes          device, [rows][K/2] packed codes (even k in the low nibble)
+ *   scales         device, [rows][K/16] E4M3 bytes, or NULL
+ *   scales_packed  device, nvfp4_scale_layout_bytes(rows, K) bytes in the MMA
+ *                  layout of nvfp4_pack_scales (rows past `rows` zero), or
+ *                  NULL; needs K % 64 == 0
+ *   g_out          device, one float: g (the per-tensor scale to pass as gA)
+ *   workspace      device scratch of NVFP4_QUANTIZE_WORKSPACE_BYTES bytes,
+ *                  caller-owned; the call clears it itself (so it needs no
+ *                  initialisation), and calls that share one must not overlap
+ * At least one of scales / scales_packed.  K % 16 == 0, rows >= 0 (rows == 0
+ * writes g = 1 only).  All buffers 16-byte aligned, g_out 4-byte aligned.
+ * Asynchronous on `stream` (one memset and two kernels); the result is
+ * deterministic.  Errors as the other entry points. */
+NVFP4_API nvfp4_status nvfp4_quantize_bf16(const void* X_bf16, int rows, int K, uint8_t* codes,
+                                           uint8_t* scales, uint8_t* scales_packed, float* g_out,
+                                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* gemm_nvfp4_w4a4 with both scale matrices already packed
  * (nvfp4_pack_scales).  Runs on pairs of SMs (tcgen05 cta_group::2, 256 x 256
  * tiles) and moves the packed scales with plain TMA tile loads, so no scale

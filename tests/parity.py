@@ -31,3 +31,14 @@ def check(y, ref, what=""):
     assert rel <= REL_FRO_TOL, f"{what}: relative Frobenius error {rel:.3e} > {REL_FRO_TOL}"
     assert mx <= MAX_ABS_REL_TOL, f"{what}: max |err|/max|ref| {mx:.3e} > {MAX_ABS_REL_TOL}"
     return rel, mx
+
+
+def packed_reference(s, K):
+    """The MMA scale layout restated: packed[rb][ks][i][j][t] = s[rb*128 + 32j + i][4ks + t],
+    zero rows past the end (numpy reshapes only)."""
+    rows = s.shape[0]
+    rb_n = (rows + 127) // 128
+    pad = np.zeros((rb_n * 128, K // 16), np.uint8)
+    pad[:rows] = s
+    v = pad.reshape(rb_n, 4, 32, K // 64, 4)          # [rb][j][i][ks][t]
+    return np.ascontiguousarray(v.transpose(0, 3, 2, 1, 4)).ravel()  # [rb][ks][i][j][t]

@@ -7,23 +7,13 @@ import oracle
 import block_scaled_precision_nvfp4_b200 as nv
 from block_scaled_precision_nvfp4_b200 import workloads as wl
 
-from parity import bf16_to_f64, check
+from parity import bf16_to_f64, check, packed_reference
 
 pytestmark = pytest.mark.gpu
 
 
 def _dev(x):
     return torch.from_numpy(np.ascontiguousarray(x)).cuda()
-
-
-def packed_reference(s, K):
-    """packed[rb][ks][i][j][t] = s[rb*128 + 32j + i][4ks + t], zero rows past the end."""
-    rows = s.shape[0]
-    rb_n = (rows + 127) // 128
-    pad = np.zeros((rb_n * 128, K // 16), np.uint8)
-    pad[:rows] = s
-    v = pad.reshape(rb_n, 4, 32, K // 64, 4)          # [rb][j][i][ks][t]
-    return np.ascontiguousarray(v.transpose(0, 3, 2, 1, 4)).ravel()  # [rb][ks][i][j][t]
 
 
 @pytest.mark.parametrize("rows,K", [(1, 64), (128, 256), (130, 512), (300, 1024), (4096, 14336),

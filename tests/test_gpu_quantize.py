@@ -1,0 +1,140 @@
+"""GPU NVFP4 activation quantiser: bit-exact against the oracle's quantiser, through the C ABI.
+
+Codes, scale bytes, the packed scale layout and g are integer / byte / exact
+results, so every comparison is exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import quantize as oq
+import block_scaled_precision_nvfp4_b200 as nv
+
+from parity import bf16_to_f64, check, packed_reference
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(x):
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _gpu(bits, plain=True, packed=True):
+    x = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    codes, s, sp, g = nv.nvfp4_quantize_bf16(x, plain=plain, packed=packed)
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    return (codes.cpu().numpy(), None if s is None else s.cpu().numpy(),
+            None if sp is None else sp.cpu().numpy(), float(g.cpu().numpy()[0]))
+
+
+def _expect_equal(bits, K, plain=True, packed=True):
+    c, s, sp, g = _gpu(bits, plain, packed)
+    rc, rs, rg = oq.quantize_nvfp4_bf16(bits)
+    assert g == float(rg)
+    assert np.array_equal(c, rc), f"codes differ at {np.argwhere(c != rc)[:5]}"
+    if plain:
+        assert np.array_equal(s, rs), f"scales differ at {np.argwhere(s != rs)[:5]}"
+    if packed:
+        ref = packed_reference(rs, K)
+        assert np.array_equal(sp[:ref.size], ref)
+
+
+SHAPES = [(1, 16), (3, 48), (1, 64), (130, 320), (128, 256), (257, 1024), (64, 4160),
+          (1000, 2048)]
+
+
+@pytest.mark.parametrize("rows,K", SHAPES)
+def test_random_shapes_bit_exact(rows, K):
+    rng = np.random.default_rng(rows * 7919 + K)
+    bits = _bits(rng.standard_normal((rows, K)).astype(np.float32) * np.float32(rng.uniform(0.01, 30)))
+    _expect_equal(bits, K, plain=True, packed=(K % 64 == 0))
+
+
+def test_plain_only_and_packed_only():
+    rng = np.random.default_rng(1)
+    bits = _bits(rng.standard_normal((200, 512)).astype(np.float32))
+    _expect_equal(bits, 512, plain=True, packed=False)
+    _expect_equal(bits, 512, plain=False, packed=True)
+
+
+def test_special_values():
+    """Zero rows and blocks, -0, tiny values that give E4M3-subnormal and zero block
+    scales, the BF16 extremes, and values at E2M1 midpoints of their block."""
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((8, 256)).astype(np.float32)
+    x[0] = 0.0                                  # a zero row
+    x[1, :16] = -0.0                            # a block of -0
+    x[2, 16:32] = 1e-30                         # underflows to a zero scale against the amax
+    x[3, :16] = np.float32(3e38)                # the tensor amax near the BF16 maximum
+    x[3, 16:32] = -np.float32(3e38)
+    x[4, 32:48] = np.float32(1e-5) * rng.standard_normal(16)   # subnormal E4M3 scales
+    base = np.float32(2.0 ** -3)
+    x[5, :16] = base * np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -0.25, -0.75,
+                                 -1.25, -1.75, -2.5, -3.5, -5, 0], np.float32)
+    _expect_equal(_bits(x), 256)
+
+
+def test_all_zero_tensor_and_empty():
+    _expect_equal(np.zeros((4, 64), np.uint16), 64)
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    codes, s, sp, g = nv.nvfp4_quantize_bf16(x)
+    torch.cuda.synchronize()
+    assert codes.numel() == 0 and float(g.cpu()[0]) == 1.0
+
+
+def test_ffn_down_activations_full_size_sampled():
+    """The FFN-down activations (4096 x 14336, N(0,1)): the whole GPU result against the
+    oracle on sampled rows, with the tensor's amax."""
+    rng = np.random.default_rng(0)
+    M, K = 4096, 14336
+    xb = _bits(rng.standard_normal((M, K), dtype=np.float32))
+    c, s, sp, g = _gpu(xb)
+    amax = np.max(np.abs(oq.bf16_to_f32(xb)))
+    rows = np.concatenate([np.arange(4), rng.choice(M, 60, replace=False), [M - 1]])
+    rc, rs, rg = oq.quantize_nvfp4_bf16(xb[rows], amax=amax)
+    assert g == float(rg)
+    assert np.array_equal(c[rows], rc) and np.array_equal(s[rows], rs)
+    ref = packed_reference(s, K)       # the packed copy holds exactly the plain bytes
+    assert np.array_equal(sp[:ref.size], ref)
+
+
+def test_quantised_activations_feed_the_w4a4_product():
+    """GPU quantiser -> packed W4A4 product: the result matches the oracle's product of
+    the same bytes (the quantiser's packed scales are consumed as they are)."""
+    rng = np.random.default_rng(3)
+    M, N, K = 300, 256, 1024
+    xb = _bits(rng.standard_normal((M, K), dtype=np.float32))
+    x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+    codes, s, sp, g = nv.nvfp4_quantize_bf16(x)
+    from block_scaled_precision_nvfp4_b200 import workloads as wl
+    W = wl.quantize_nvfp4(rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02))
+    wd = torch.from_numpy(W.codes).cuda()
+    swp = nv.nvfp4_pack_scales(torch.from_numpy(W.scales).cuda(), K)
+    gA = float(g.cpu()[0])
+    y = nv.gemm_nvfp4_w4a4_packed(codes, sp, gA, wd, swp, W.g)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_w4a4(codes.cpu().numpy(), s.cpu().numpy(), gA, W.codes, W.scales, W.g, M, N, K)
+    check(bf16_to_f64(y), ref, "quantise -> W4A4")
+
+
+def test_repeat_is_deterministic_and_workspace_reusable():
+    rng = np.random.default_rng(4)
+    bits = _bits(rng.standard_normal((256, 512)).astype(np.float32))
+    x = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    ws = torch.full((16,), 0xAB, dtype=torch.uint8, device="cuda")   # garbage: the call clears it
+    a = nv.nvfp4_quantize_bf16(x, workspace=ws)
+    b = nv.nvfp4_quantize_bf16(x, workspace=ws)
+    torch.cuda.synchronize()
+    assert all(torch.equal(p, q) for p, q in zip(a, b))
+
+
+def test_argument_errors():
+    x = torch.zeros((4, 40), dtype=torch.bfloat16, device="cuda")   # K % 16 != 0
+    with pytest.raises(nv.NvFp4Error) as e:
+        nv.nvfp4_quantize_bf16(x)
+    assert e.value.status == nv.Status.INVALID_ARG
+    x = torch.zeros((4, 48), dtype=torch.bfloat16, device="cuda")   # packed needs K % 64
+    with pytest.raises(nv.NvFp4Error) as e:
+        nv.nvfp4_quantize_bf16(x, packed=True)
+    assert e.value.status == nv.Status.INVALID_ARG
