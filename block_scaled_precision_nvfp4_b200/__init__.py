@@ -94,6 +94,7 @@ C_FUNCTIONS = {
     "gemm_nvfp4_w4a4_grouped_packed": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
     "nvfp4_quantize_workspace_bytes": (_Z, []),
     "nvfp4_quantize_bf16": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "nvfp4_quantize_bf16_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _P]),
 }
 
 _lock = threading.Lock()

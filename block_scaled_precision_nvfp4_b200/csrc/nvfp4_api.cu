@@ -470,6 +470,63 @@ nvfp4_status nvfp4_quantize_bf16(const void* X, int rows, int K, uint8_t* codes,
     return ok();
 }
 
+// ------------------------------------------------------------------------- quantiser without
+// a caller workspace
+//
+// nvfp4_quantize_bf16 keeps its running amax in a few bytes of caller-owned
+// device scratch.  This variant keeps them in a static device array instead, so
+// a caller that cannot allocate device memory (or cannot keep a scratch buffer
+// between calls) can still quantise.  The array lives in every GPU that loads
+// the library until the process exits; its device address is looked up once
+// per device.
+namespace {
+constexpr size_t kNoAllocScratchBytes = 256;  // the stated maximum; the quantiser needs 16
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+static_assert(NVFP4_QUANTIZE_WORKSPACE_BYTES <= kNoAllocScratchBytes,
+              "the static scratch must hold the quantiser's workspace");
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// The device address of g_noalloc_scratch on the current device (the host-side
+// name is only a stand-in for it), looked up on the first call per device.
+nvfp4_status noalloc_scratch(int dev, void** out) {
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(NVFP4_ERR_CUDA, "device %d is beyond the %d devices this entry point tracks", dev,
+                    kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "looking up the static quantiser scratch");
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return NVFP4_OK;
+}
+}  // namespace
+
+nvfp4_status nvfp4_quantize_bf16_noalloc(const void* X, int rows, int K, uint8_t* codes,
+                                         uint8_t* scales, uint8_t* scales_packed, float* g_out,
+                                         void* stream) {
+    const size_t need = nvfp4_quantize_workspace_bytes();  // does not grow with the tensor
+    if (need > kNoAllocScratchBytes)
+        return fail(NVFP4_ERR_INVALID_ARG,
+                    "this call needs %zu bytes of scratch, more than the %zu of the static array",
+                    need, kNoAllocScratchBytes);
+    int dev;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(NVFP4_ERR_CUDA, "cannot query the current CUDA device");
+    }
+    void* scratch = nullptr;
+    nvfp4_status st = noalloc_scratch(dev, &scratch);
+    if (st != NVFP4_OK) return st;
+    return nvfp4_quantize_bf16(X, rows, K, codes, scales, scales_packed, g_out, scratch,
+                               kNoAllocScratchBytes, stream);
+}
+
 nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, float gA,
                                     const uint8_t* W, const uint8_t* sW_packed, float gW,
                                     void* Y, int M, int N, int K, void* stream) {

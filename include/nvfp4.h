@@ -186,6 +186,29 @@ NVFP4_API nvfp4_status nvfp4_quantize_bf16(const void* X_bf16, int rows, int K, 
                                            uint8_t* scales, uint8_t* scales_packed, float* g_out,
                                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* nvfp4_quantize_bf16 for callers that cannot allocate device memory: the
+ * same operation, arguments (minus the workspace), results and errors, with
+ * the few bytes of scratch it needs kept in a static device array of 256 bytes
+ * inside the library instead of a caller buffer.  It is meant for code that may
+ * not call cudaMalloc at all -- for example code that runs after an inference
+ * runtime has handed all device memory to its own pool, or a plugin whose
+ * enqueue step must not allocate -- and for callers with nowhere to keep a
+ * scratch buffer between calls.  This entry point has no counterpart on the
+ * pages; it is a convenience of this library.
+ *   - It allocates nothing and calls no allocating routine.  Every GPU that
+ *     loads the library holds the 256-byte array until the process exits.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device); make that first call before any stream capture.
+ *   - Every call uses the same array; the call clears the part it needs, but
+ *     calls whose work overlaps on the GPU (other streams, other threads) race
+ *     on it and must be ordered by the caller.
+ *   - The scratch it needs does not grow with the tensor; a need beyond the
+ *     array's 256 bytes is refused with NVFP4_ERR_INVALID_ARG. */
+NVFP4_API nvfp4_status nvfp4_quantize_bf16_noalloc(const void* X_bf16, int rows, int K,
+                                                   uint8_t* codes, uint8_t* scales,
+                                                   uint8_t* scales_packed, float* g_out,
+                                                   void* stream);
+
 /* gemm_nvfp4_w4a4 with both scale matrices already packed
  * (nvfp4_pack_scales).  Runs on pairs of SMs (tcgen05 cta_group::2, 256 x 256
  * tiles) and moves the packed scales with plain TMA tile loads, so no scale
