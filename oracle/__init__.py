@@ -10,8 +10,8 @@ module doc (bullets 1 and 2): the NVFP4 block-scaled product
 
     Y[m,n] = gA*gW * sum_g sA[m,g]*sW[n,g] * sum_{k in g} e2m1(A[m,k])*e2m1(W[n,k])
 
-and its two sibling paths (the exact E2M1->E4M3 FP8 path and the BF16-widen
-W4A16 path).  Layouts: packed codes ``uint8[rows, K/2]`` (even k in the low
+and its sibling paths (the exact E2M1->E4M3 FP8 path, the BF16-widen W4A16
+path, and W4A8: FP8 activations under NVFP4 weights on the exact E4M3 path).  Layouts: packed codes ``uint8[rows, K/2]`` (even k in the low
 nibble), E4M3 scales ``uint8[rows, K/16]``, BF16 as ``uint16`` bits.
 """
 from __future__ import annotations
@@ -61,6 +61,11 @@ def _load():
                                ("oracle_gemm_via_fp8", dense), ("oracle_gemm_via_fp8_at", at)):
                 getattr(lib, name).argtypes = args
                 getattr(lib, name).restype = ctypes.c_int
+            lib.oracle_gemm_w4a8.argtypes = [P, D, P, P, D, I64, I64, I64, P, ctypes.c_int]
+            lib.oracle_gemm_w4a8.restype = ctypes.c_int
+            lib.oracle_gemm_w4a8_at.argtypes = [P, D, P, P, D, I64, I64, I64, P, P, I64, P,
+                                                ctypes.c_int]
+            lib.oracle_gemm_w4a8_at.restype = ctypes.c_int
             lib.oracle_gemm_w4a16.argtypes = [P, P, P, D, I64, I64, I64, P, ctypes.c_int]
             lib.oracle_gemm_w4a16.restype = ctypes.c_int
             lib.oracle_gemm_w4a16_at.argtypes = [P, P, P, D, I64, I64, I64, P, P, I64, P,
@@ -149,6 +154,24 @@ def _dense_or_at(name, A, sA, gA, W, sW, gW, M, N, K, rows, cols, threads):
     out = np.empty(r.shape, dtype=np.float64)
     _check(getattr(lib, name + "_at")(_ptr(A), _ptr(sA), float(gA), _ptr(W), _ptr(sW),
                                       float(gW), M, N, K, _ptr(r), _ptr(c), r.size, _ptr(out), t))
+    return out
+
+
+def gemm_w4a8(A_fp8, gA, W, sW, gW, M, N, K, rows=None, cols=None, threads=None):
+    """FP64 W4A8: E4M3 activation bytes [M,K] (per-tensor scale gA) times NVFP4 W."""
+    lib = _load()
+    t = threads or default_threads()
+    A = _u8(A_fp8, (M, K))
+    W = _u8(W, (N, K // 2)); sW = _u8(sW, (N, K // 16))
+    if rows is None:
+        Y = np.empty((M, N), dtype=np.float64)
+        _check(lib.oracle_gemm_w4a8(_ptr(A), float(gA), _ptr(W), _ptr(sW), float(gW), M, N, K,
+                                    _ptr(Y), t))
+        return Y
+    r, c = _pairs(rows, cols)
+    out = np.empty(r.shape, dtype=np.float64)
+    _check(lib.oracle_gemm_w4a8_at(_ptr(A), float(gA), _ptr(W), _ptr(sW), float(gW), M, N, K,
+                                   _ptr(r), _ptr(c), r.size, _ptr(out), t))
     return out
 
 

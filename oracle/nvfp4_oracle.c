@@ -162,11 +162,31 @@ static double elem_w4a16(const uint16_t* A, const uint8_t* W, const uint8_t* sW,
     return gW * acc;
 }
 
+/* W4A8: FP8 (E4M3) activations under NVFP4 weights (module doc, exec_of:
+ * "W4A8 with group-16 E4M3 scales ... take the exact E4M3 path").  The
+ * activations carry only their per-tensor scale gA; the weights their group
+ * scales and gW:  Y = gA*gW * sum_g sW[n,g] * sum_{k in g} e4m3(A[m,k]) * e2m1(W[n,k]).
+ * A is one E4M3 byte per element [M][K]; NaN bytes (0x7F, 0xFF) are not inputs. */
+static double elem_w4a8(const uint8_t* A, const uint8_t* W, const uint8_t* sW, double alpha,
+                        int64_t K, int64_t m, int64_t n) {
+    const int64_t G = K / 16;
+    const uint8_t* a = A + m * K;
+    const uint8_t* w = W + n * (K / 2);
+    double acc = 0.0;
+    for (int64_t g = 0; g < G; ++g) {
+        double p = 0.0; /* exact: 16 products on a 2^-10 grid, |p| <= 16 * 448 * 6 */
+        for (int64_t k = 16 * g; k < 16 * g + 16; ++k)
+            p += e4m3(a[k]) * E2M1[code_at(w, k)];
+        acc += e4m3(sW[n * G + g]) * p;
+    }
+    return alpha * acc;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Threaded drivers over a list of output elements                            */
 /* ------------------------------------------------------------------------- */
 
-enum { P_W4A4 = 0, P_VIA_FP8 = 1, P_W4A16 = 2, P_GROUPED = 3 };
+enum { P_W4A4 = 0, P_VIA_FP8 = 1, P_W4A16 = 2, P_GROUPED = 3, P_W4A8 = 4 };
 
 typedef struct {
     int path;
@@ -200,6 +220,8 @@ static double one(const job_t* j, int64_t m, int64_t n) {
         return elem_via_fp8((const uint8_t*)j->A, j->sA, j->W, j->sW, j->gA * j->gW, j->K, m, n);
     case P_W4A16:
         return elem_w4a16((const uint16_t*)j->A, j->W, j->sW, j->gW, j->K, m, n);
+    case P_W4A8:
+        return elem_w4a8((const uint8_t*)j->A, j->W, j->sW, j->gA * j->gW, j->K, m, n);
     case P_GROUPED: {
         int64_t e = expert_of(j->offsets, j->E, m);
         const uint8_t* We = j->W + e * j->N * (j->K / 2);
@@ -280,6 +302,21 @@ int oracle_gemm_via_fp8_at(const uint8_t* A, const uint8_t* sA, double gA, const
                            double* out, int nthreads) {
     if (bad_shape(M, N, K)) return -2;
     job_t j = {P_VIA_FP8, A, sA, W, sW, gA, gW, NULL, NULL, 0, M, N, K, rows, cols, count, out, 0, 0};
+    return run(j, nthreads);
+}
+
+int oracle_gemm_w4a8(const uint8_t* A, double gA, const uint8_t* W, const uint8_t* sW, double gW,
+                     int64_t M, int64_t N, int64_t K, double* Y, int nthreads) {
+    if (bad_shape(M, N, K)) return -2;
+    job_t j = {P_W4A8, A, NULL, W, sW, gA, gW, NULL, NULL, 0, M, N, K, NULL, NULL, M * N, Y, 0, 0};
+    return run(j, nthreads);
+}
+
+int oracle_gemm_w4a8_at(const uint8_t* A, double gA, const uint8_t* W, const uint8_t* sW,
+                        double gW, int64_t M, int64_t N, int64_t K, const int64_t* rows,
+                        const int64_t* cols, int64_t count, double* out, int nthreads) {
+    if (bad_shape(M, N, K)) return -2;
+    job_t j = {P_W4A8, A, NULL, W, sW, gA, gW, NULL, NULL, 0, M, N, K, rows, cols, count, out, 0, 0};
     return run(j, nthreads);
 }
 
