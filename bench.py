@@ -69,6 +69,8 @@ def peaks():
 WORKLOADS = {
     "ffn_down": dict(path="w4a4", bound="tensor", desc="FFN down W4A4 4096x5376x14336"),
     "via_fp8": dict(path="via_fp8", bound="alu", desc="FFN down through the exact FP8 path"),
+    "w4a8": dict(path="w4a8", bound="alu",
+                 desc="FFN down W4A8 (E4M3 activations) 4096x5376x14336"),
     "w4a16": dict(path="w4a16", bound="hbm", desc="W4A16 decode 16x5376x14336"),
     "grouped": dict(path="grouped", bound="tensor", desc="grouped MoE W4A4, 8 experts"),
     "tiny": dict(path="w4a4", bound="tensor", desc="tiny W4A4 128x256x256"),
@@ -87,6 +89,8 @@ def make_workload(name):
         return wl.grouped_w4a4()
     if name == "quantize":
         return wl.activations_bf16()
+    if name == "w4a8":
+        return wl.w4a8_ffn_down()
     return wl.ffn_down_w4a4()
 
 
@@ -98,7 +102,10 @@ def algorithmic(wl_, path):
     if path == "quantize":
         # X read once; codes, packed scales and g written (the two-pass amax reads X twice)
         return 0.0, M * K * 2 + M * K // 2 + M * K // 16 + 4
+    if path == "w4a16":
         return flops, N * K // 2 + N * K // 16 + M * K * 2 + ybytes
+    if path == "w4a8":
+        return flops, N * K // 2 + N * K // 16 + M * K + ybytes
     if path == "grouped":
         return flops, wl_.E * (N * K // 2 + N * K // 16) + M * (K // 2 + K // 16) + ybytes
     return flops, (M + N) * (K // 2 + K // 16) + ybytes
@@ -176,7 +183,10 @@ def _oracle_rows(wl_, rows):
         from oracle import quantize as oq
         oq.quantize_nvfp4_bf16(wl_.A_bf16[:rows])
         return
-    if wl_.A_bf16 is not None:
+    if wl_.A_fp8 is not None:
+        oracle.gemm_w4a8(wl_.A_fp8[:rows], wl_.gA, wl_.W.codes, wl_.W.scales, wl_.W.g, rows,
+                         wl_.N, wl_.K)
+    elif wl_.A_bf16 is not None:
         oracle.gemm_w4a16(wl_.A_bf16[:rows], wl_.W.codes, wl_.W.scales, wl_.W.g, rows, wl_.N,
                           wl_.K)
     elif wl_.E:
@@ -258,6 +268,7 @@ def run_reference(args):
 KERNEL_SOURCES = {
     "w4a4": ["w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
     "via_fp8": ["via_fp8_kernel.cuh", "ptx.cuh"],
+    "w4a8": ["w4a8_kernel.cuh", "via_fp8_kernel.cuh", "ptx.cuh"],
     "w4a16": ["w4a16_kernel.cuh"],
     "grouped": ["grouped_pair_kernel.cuh", "w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
     "quantize": ["quantize_kernel.cuh"],
@@ -322,6 +333,8 @@ def run_ours(args):
         host = [wl_.A_bf16.view(np.int16)]
     elif path == "w4a16":
         host = [wl_.A_bf16.view(np.int16), wl_.W.codes, wl_.W.scales]
+    elif path == "w4a8":
+        host = [wl_.A_fp8, wl_.W.codes, wl_.W.scales]
     elif path == "grouped":
         Wc, Ws, gW = wlm.stack_experts(wl_)
         host = [wl_.A.codes, wl_.A.scales, Wc, Ws]
@@ -368,6 +381,9 @@ def run_ours(args):
         def plain_step():
             nv.gemm_nvfp4_w4a4_grouped(dv[0], dv[1], wl_.A.g, dv[2], dv[3], gw_list, offs,
                                        out=Y, stream=stream)
+    elif path == "w4a8":
+        def step():
+            nv.gemm_nvfp4_w4a8(dv[0], wl_.gA, dv[1], dv[2], wl_.W.g, out=Y, stream=stream)
     elif path == "via_fp8":
         def step():
             nv.gemm_nvfp4_via_fp8(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
@@ -482,7 +498,7 @@ def run_ours(args):
                  "gemm_packed_ms": statistics.median(gemm_ms),
                  "plain_scale_entry_ms": statistics.median(plain),
                  "plain_scale_entry_tflops": flops / (statistics.median(plain) * 1e-3) / 1e12}
-    kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel",
+    kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel", "w4a8": "w4a8_kernel",
                    "w4a16": "w4a16_kernel", "grouped": "grouped_pair_kernel",
                    "quantize": "quantize_bf16_kernel (+ amax_bf16_kernel)"}[path]
     if spec["bound"] == "tensor":
@@ -519,17 +535,18 @@ def run_ours(args):
                                                        else "weight codes")
                                + " after the same flush; GB/s counts read + write")}
     else:
-        # each (row, column, group) update is two FP32 operations (the scale product
-        # and the FMA into the accumulator) on 128 FP32 lanes per SM:
-        # SMs x 64 updates per clock x max clock
+        # each (row, column, group) update is FP32 work on 128 FP32 lanes per SM: two
+        # operations on the W4A4 exact path (the scale product and the FMA into the
+        # accumulator), one on the W4A8 path (the weights' scale only: one FMA)
+        ops = 1 if path == "w4a8" else 2
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         clk_mhz = clk.summary().get("sm_max_mhz") or 1965
-        peak_upd = sms * 64 * clk_mhz * 1e6 / 1e12  # T updates / s
+        peak_upd = sms * (128 // ops) * clk_mhz * 1e6 / 1e12  # T updates / s
         achieved = (M * N * K / 16) / kern_s / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": peak_upd,
                 "unit": "Tupdate/s", "frac": achieved / peak_upd,
-                "peak_note": ("per-16 FP32 scale-apply updates, 2 FP32 ops each; derived: "
-                              "SMs x 128 FP32 lanes / 2 x max clock")}
+                "peak_note": (f"per-16 FP32 scale-apply updates, {ops} FP32 op(s) each; derived: "
+                              f"SMs x 128 FP32 lanes / {ops} x max clock")}
     roof.update({"traffic": profiled_traffic(wl_.name, path), "kernel": kernel_name,
                  "kernel_ms": kern_s * 1e3})
     roof.update(extra)
@@ -542,6 +559,8 @@ def run_ours(args):
         "dtype": ("bf16 -> nvfp4 (fp32 scale arithmetic)" if path == "quantize" else
                   "bf16 x nvfp4(e2m1, e4m3 group scales) -> f32 accumulate -> bf16"
                   if path == "w4a16" else
+                  "e4m3 x nvfp4(e2m1, e4m3 group scales) -> f32 accumulate -> bf16"
+                  if path == "w4a8" else
                   "nvfp4(e2m1 x e2m1, e4m3 group scales) -> f32 accumulate -> bf16"),
         "data": "synthetic",
         "config": {"workload": wl_.name, "M": M, "N": N, "K": K, "global_batch": world * M,

@@ -25,7 +25,7 @@ __all__ = [
     "Fmt", "Kind", "Exec", "Status", "NvFp4Error", "load_library", "library_path",
     "nvfp4_kind_of", "nvfp4_exec_of", "nvfp4_exec_of_arch", "nvfp4_pair_name",
     "nvfp4_exec_name", "nvfp4_set_fp4_kernel_disabled", "nvfp4_version",
-    "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_w4a16",
+    "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_nvfp4_w4a8", "gemm_w4a16",
     "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
     "gemm_nvfp4_w4a4_packed", "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
     "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "C_FUNCTIONS",
@@ -84,6 +84,7 @@ C_FUNCTIONS = {
     "nvfp4_check_device_error": (_I, [_P]),
     "gemm_nvfp4_w4a4": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_nvfp4_via_fp8": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
+    "gemm_nvfp4_w4a8": (_I, [_P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
     "nvfp4_scale_layout_bytes": (_Z, [_I, _I]),
     "nvfp4_pack_scales": (_I, [_P, _I, _I, _P, _P]),
     "gemm_nvfp4_w4a4_packed": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
@@ -306,6 +307,24 @@ def gemm_nvfp4_w4a4_packed(A, sA_packed, gA, W, sW_packed, gW, out=None, stream=
 def gemm_nvfp4_via_fp8(A, sA, gA, W, sW, gW, out=None, stream=None):
     """The same product through the exact E2M1->E4M3 conversion on the FP8 MMA."""
     return _w4a4_common("gemm_nvfp4_via_fp8", A, sA, gA, W, sW, gW, out, stream)
+
+
+def gemm_nvfp4_w4a8(A_fp8, gA, W, sW, gW, out=None, stream=None):
+    """Y[M,N] (bf16) = gA*gW * A_fp8 . (W.sW)^T: E4M3 activation bytes [M,K] under NVFP4
+    weights, on the exact E4M3 path (K % 256 == 0)."""
+    torch = _torch()
+    M, K = A_fp8.shape
+    N = W.shape[0]
+    a = A_fp8.view(torch.uint8) if A_fp8.dtype != torch.uint8 else A_fp8
+    pa = _dev_tensor(a, torch.uint8, (M, K), "A_fp8")
+    pw = _dev_tensor(W, torch.uint8, (N, K // 2), "W")
+    psw = _dev_tensor(sW, torch.uint8, (N, K // 16), "sW")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A_fp8.device)
+    py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
+    _err(load_library().gemm_nvfp4_w4a8(pa, float(gA), pw, psw, float(gW), py, M, N, K,
+                                        _stream_ptr(stream)))
+    return out
 
 
 def gemm_w4a16(A, W, sW, gW, out=None, stream=None):

@@ -21,6 +21,7 @@
 #include "pack_scales_kernel.cuh"
 #include "w4a16_kernel.cuh"
 #include "via_fp8_kernel.cuh"
+#include "w4a8_kernel.cuh"
 #include "grouped_kernel.cuh"
 #include "grouped_pair_kernel.cuh"
 #include "quantize_kernel.cuh"
@@ -317,7 +318,9 @@ nvfp4_exec nvfp4_exec_of_arch(int arch, nvfp4_fmt weight, nvfp4_fmt activation,
     case NVFP4_KIND_BF16_MMA:
         return class_compiles_bf16_widen_kernel(arch) ? NVFP4_EXEC_BF16_WIDEN : NVFP4_EXEC_NO_PATH;
     case NVFP4_KIND_FP8_MMA:
-        // W4A8 has no single-instruction MMA; its exact E4M3 path is not carried yet.
+        // W4A8 has no single-instruction MMA (no FP4 x FP8 MMA takes E4M3 group-16
+        // scales); it takes the exact E4M3 path where that kernel is compiled.
+        if (class_has_fp8_mma(arch) && class_compiles_fp8_exact_kernel(arch)) return NVFP4_EXEC_FP8_EXACT;
         return NVFP4_EXEC_NO_PATH;
     default:
         return NVFP4_EXEC_NO_PATH;
@@ -608,6 +611,43 @@ nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, float gA, c
         tmA, tmB, tmSA, tmSB, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launching via_fp8_kernel");
+    return ok();
+}
+
+// ------------------------------------------------------------------------- W4A8
+nvfp4_status gemm_nvfp4_w4a8(const uint8_t* A_fp8, float gA, const uint8_t* W, const uint8_t* sW,
+                             float gW, void* Y, int M, int N, int K, void* stream) {
+    namespace k8 = nvfp4::w4a8;
+    if (M < 0 || N < 0) return fail(NVFP4_ERR_INVALID_ARG, "M and N must be >= 0 (got %d, %d)", M, N);
+    if (K < k8::BK || K % k8::BK != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "W4A8 needs K a positive multiple of 256 (got %d)", K);
+    if (M > 0 && N > 0) {
+        if (!A_fp8 || !W || !sW || !Y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+        if (!aligned16(A_fp8) || !aligned16(W) || !aligned16(sW) || !aligned16(Y))
+            return fail(NVFP4_ERR_MISALIGNED, "every buffer must be 16-byte aligned");
+    }
+    int dev;
+    DevInfo info;
+    if (!current_device(dev, info)) return fail(NVFP4_ERR_CUDA, "cannot query the current CUDA device");
+    if (nvfp4_exec_of_arch(info.sm_arch, NVFP4_FMT_NVFP4, NVFP4_FMT_FP8_E4M3, 0) != NVFP4_EXEC_FP8_EXACT)
+        return fail(NVFP4_ERR_NOPATH, "no exact E4M3-path kernel for W4A8 is compiled for sm_%d",
+                    info.sm_arch);
+    if (M == 0 || N == 0) return ok();
+
+    nvfp4_status st;
+    CUtensorMap tmA, tmB, tmSB;
+    if ((st = make_map_u8(&tmA, A_fp8, (uint64_t)K, (uint64_t)M, 128, k8::BM)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmB, W, (uint64_t)K / 2, (uint64_t)N, 128, k8::BN)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmSB, sW, (uint64_t)K / 16, (uint64_t)N, 16, k8::BN,
+                          CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
+        return st;
+    if ((st = set_smem(k8::w4a8_kernel, k8::SMEM_BYTES, info, "w4a8_kernel")) != NVFP4_OK) return st;
+    const int tiles = ((M + k8::BM - 1) / k8::BM) * ((N + k8::BN - 1) / k8::BN);
+    const int grid = tiles < info.num_sms ? tiles : info.num_sms;
+    k8::w4a8_kernel<<<grid, k8::NUM_THREADS, k8::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
+        tmA, tmB, tmSB, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launching w4a8_kernel");
     return ok();
 }
 

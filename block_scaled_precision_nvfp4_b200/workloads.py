@@ -46,6 +46,8 @@ class Workload:
     A: Operand | None = None          # NVFP4 activations (W4A4 paths)
     W: Operand | None = None          # NVFP4 weights [N, K]
     A_bf16: np.ndarray | None = None  # uint16 BF16 bit patterns [M, K] (W4A16)
+    A_fp8: np.ndarray | None = None   # uint8 E4M3 bytes [M, K] (W4A8)
+    gA: float = 1.0                   # FP32 per-tensor scale of A_fp8
     # grouped
     E: int = 0
     offsets: np.ndarray | None = None  # int64 [E+1]
@@ -200,6 +202,37 @@ def activations_bf16(M: int = 4096, K: int = 14336, seed: int = 0) -> Workload:
     A = to_bf16_bits(rng.standard_normal((M, K), dtype=np.float32))
     return Workload(f"quantize_bf16_{M}x{K}", M, 0, K, A_bf16=A,
                     notes="X bf16 N(0,1) seed %d" % seed)
+
+
+def fp8_per_tensor(rng: np.random.Generator, rows: int, K: int, std: float = 1.0,
+                   chunk_rows: int = 2048) -> tuple[np.ndarray, float]:
+    """N(0, std) [rows, K] as E4M3 bytes with one FP32 per-tensor scale gA = amax/448
+    (x / gA rounded to nearest even by torch's cast), drawn in row chunks."""
+    state = rng.bit_generator.state
+    amax = 0.0
+    for r0 in range(0, rows, chunk_rows):
+        r1 = min(rows, r0 + chunk_rows)
+        amax = max(amax, float(np.max(np.abs(
+            rng.standard_normal((r1 - r0, K), dtype=np.float32) * np.float32(std)))))
+    rng.bit_generator.state = state
+    g = np.float32(amax / E4M3_MAX) if amax > 0 else np.float32(1.0)
+    out = np.empty((rows, K), dtype=np.uint8)
+    for r0 in range(0, rows, chunk_rows):
+        r1 = min(rows, r0 + chunk_rows)
+        x = rng.standard_normal((r1 - r0, K), dtype=np.float32) * np.float32(std)
+        out[r0:r1] = e4m3_rne(x / g)
+    return out, float(g)
+
+
+def w4a8_ffn_down(M: int = 4096, N: int = 5376, K: int = 14336, seed_a: int = 0,
+                  seed_w: int = 1) -> Workload:
+    """FFN down projection with FP8 activations: A ~ N(0,1) [M,K] (seed 0) as E4M3 bytes
+    with a per-tensor scale; W as the FFN-down NVFP4 weights (seed 1)."""
+    A8, gA = fp8_per_tensor(np.random.Generator(np.random.PCG64(seed_a)), M, K)
+    W = quantize_nvfp4_chunked(np.random.Generator(np.random.PCG64(seed_w)), N, K, 0.02)
+    return Workload(f"w4a8_ffn_down_{M}x{N}x{K}", M, N, K, W=W, A_fp8=A8, gA=gA,
+                    notes="A e4m3 N(0,1)/gA seed %d, gA=amax/448; W~N(0,0.02) seed %d" % (
+                        seed_a, seed_w))
 
 
 def zipf_routing(tokens: int, E: int, s: float, seed: int) -> np.ndarray:

@@ -78,7 +78,7 @@ typedef enum {
 /* How a device executes a declared (weight, activation) pair (`enum Exec`). */
 typedef enum {
     NVFP4_EXEC_FP4_MMA = 0,        /* block-scaled FP4 MMA: gemm_nvfp4_w4a4 */
-    NVFP4_EXEC_FP8_EXACT = 1,      /* exact E2M1->E4M3 conversion on the FP8 MMA: gemm_nvfp4_via_fp8 */
+    NVFP4_EXEC_FP8_EXACT = 1,      /* exact E2M1->E4M3 conversion on the FP8 MMA: gemm_nvfp4_via_fp8 (W4A4), gemm_nvfp4_w4a8 (W4A8) */
     NVFP4_EXEC_BF16_WIDEN = 2,     /* BF16 MMA, NVFP4 weights widened in registers: gemm_w4a16 */
     NVFP4_EXEC_NO_FP4_KERNEL = 3,  /* device has the FP4 MMA, but its class has no compiled kernel */
     NVFP4_EXEC_NO_PATH = 4         /* neither native nor exact: refused, never widened */
@@ -97,8 +97,9 @@ NVFP4_API nvfp4_kind nvfp4_kind_of(nvfp4_fmt activation);
  * but with the FP8 MMA for which this library compiles the exact-path kernel
  * (none besides sm_100, so NO_PATH on sm_89/sm_90), NO_PATH otherwise.
  * (NVFP4, BF16): BF16_WIDEN on sm_100, NO_PATH elsewhere.
- * (NVFP4, FP8) (W4A8): no single-instruction MMA; the exact E4M3 path, which
- * this library does not carry yet, so NO_PATH.
+ * (NVFP4, FP8) (W4A8): no single-instruction MMA takes FP8 activations under
+ * NVFP4 weights with E4M3 group-16 scales, so the exact E4M3 path: FP8_EXACT on
+ * sm_100 (gemm_nvfp4_w4a8), NO_PATH on every other class.
  * Pairs whose weights are not NVFP4: NO_PATH (this library carries NVFP4-weight
  * paths only).  `fp4_kernel_disabled` != 0 behaves as if the class compiled no
  * FP4 block-scale kernel (module doc, `fp4_fallback`, `avail::without_fp4_kernel`). */
@@ -230,14 +231,31 @@ NVFP4_API nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, f
                                 const uint8_t* W, const uint8_t* sW, float gW,
                                 void* Y_bf16, int M, int N, int K, void* stream);
 
+/* W4A8: FP8 (E4M3) activations under NVFP4 weights (metrale_circuit
+ * `hardware::exec`, exec_of: W4A8 with group-16 E4M3 scales takes the exact
+ * E4M3 path):
+ *     Y[m,n] = BF16( gA*gW * sum_g sW[n,g] * sum_{k in g} a[m,k]*w[n,k] )
+ * with a[m,k] the E4M3 value of byte A_fp8[m][k] (row-major [M][K], one byte per
+ * element, any finite E4M3 byte; gA is its FP32 per-tensor scale) and W, sW, gW
+ * as for gemm_nvfp4_w4a4 (the activations carry no group scales).  The weight
+ * codes are converted by the exact E2M1 -> E4M3 identity and each 16-group's
+ * FP8 partial sum is scaled in FP32 by sW*2^6 and accumulated in FP32.
+ * M, N >= 0 (0 returns OK and does nothing); K >= 256, K % 256 == 0; every
+ * pointer a 16-byte aligned device pointer.  Needs exec_of(device, NVFP4, FP8)
+ * == FP8_EXACT (sm_100), else NVFP4_ERR_NOPATH. */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a8(const uint8_t* A_fp8, float gA, const uint8_t* W,
+                                       const uint8_t* sW, float gW, void* Y_bf16, int M, int N,
+                                       int K, void* stream);
+
 /* W4A16: BF16 activations A_bf16 [M][K] (row-major) times NVFP4 weights, the
  * weights widened to BF16 in registers (exactly: an E2M1 value times an E4M3
  * scale has at most 6 significant bits), FP32 accumulation, gW applied in the
  * epilogue, BF16 output Y [M][N].  Built for the memory-bound decode shape:
  * one launch covers 16 tokens (larger M runs as consecutive 16-token launches,
- * each re-reading W).  K is split across an 8-CTA cluster and the partial sums
- * are reduced on chip in a fixed order, so the call needs no workspace and is
- * deterministic.  M, N >= 0; K >= 32, K % 32 == 0. */
+ * each re-reading W).  One wave of CTAs, each owning a range of weight rows over
+ * the whole of K; K is split across the CTA's warps and their partial sums are
+ * added in shared memory in a fixed order, so the call needs no workspace and
+ * is deterministic.  M, N >= 0; K >= 32, K % 32 == 0. */
 NVFP4_API nvfp4_status gemm_w4a16(const void* A_bf16, const uint8_t* W, const uint8_t* sW, float gW,
                         void* Y_bf16, int M, int N, int K, void* stream);
 

@@ -64,8 +64,13 @@ def test_exec_of_other_pairs():
     F, E = nv.Fmt, nv.Exec
     assert nv.nvfp4_exec_of_arch(100, F.NVFP4, F.BF16) == E.BF16_WIDEN
     assert nv.nvfp4_exec_of_arch(90, F.NVFP4, F.BF16) == E.NO_PATH
-    # W4A8: no single-instruction MMA; its exact path is not carried -> no path, never widened
-    assert nv.nvfp4_exec_of_arch(100, F.NVFP4, F.FP8_E4M3) == E.NO_PATH
+    # W4A8: no single-instruction MMA; the exact E4M3 path where its kernel is compiled
+    # (sm_100), no path elsewhere, never widened to BF16
+    assert nv.nvfp4_exec_of_arch(100, F.NVFP4, F.FP8_E4M3) == E.FP8_EXACT
+    for arch in (89, 90, 103, 120, 80):
+        assert nv.nvfp4_exec_of_arch(arch, F.NVFP4, F.FP8_E4M3) == E.NO_PATH
+    # the FP4-kernel switch concerns the FP4 MMA only
+    assert nv.nvfp4_exec_of_arch(100, F.NVFP4, F.FP8_E4M3, fp4_kernel_disabled=True) == E.FP8_EXACT
     for w in (F.BF16, F.FP8_E4M3):
         for a in F:
             assert nv.nvfp4_exec_of_arch(100, w, a) == E.NO_PATH
@@ -155,3 +160,16 @@ def test_grouped_pack_argument_errors_need_no_device():
     assert call([0, 4], 1, K=96) == nv.Status.INVALID_ARG
     assert call([0, 4], 1, s=8) == nv.Status.MISALIGNED
     assert call([0, 0, 0], 2) == nv.Status.OK                 # nothing to pack
+
+
+def test_w4a8_argument_errors_need_no_device():
+    lib = nv.load_library()
+    def call(A=16, W=16, sW=16, Y=16, M=4, N=4, K=256):
+        return lib.gemm_nvfp4_w4a8(A, 1.0, W, sW, 1.0, Y, M, N, K, None)
+    assert call(M=-1) == nv.Status.INVALID_ARG
+    assert call(K=128) == nv.Status.INVALID_ARG      # K % 256
+    assert call(K=384) == nv.Status.INVALID_ARG
+    assert call(K=0) == nv.Status.INVALID_ARG
+    assert call(A=0) == nv.Status.INVALID_ARG
+    assert call(sW=40) == nv.Status.MISALIGNED
+    assert call(Y=8) == nv.Status.MISALIGNED
