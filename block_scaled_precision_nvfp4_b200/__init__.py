@@ -28,7 +28,8 @@ __all__ = [
     "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_nvfp4_w4a8", "gemm_w4a16",
     "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
     "gemm_nvfp4_w4a4_packed", "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
-    "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "C_FUNCTIONS",
+    "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "nvfp4_fp4_fallback",
+    "nvfp4_node_exec", "C_FUNCTIONS",
 ]
 
 
@@ -78,6 +79,8 @@ C_FUNCTIONS = {
     "nvfp4_kind_of": (_I, [_I]),
     "nvfp4_exec_of_arch": (_I, [_I, _I, _I, _I]),
     "nvfp4_exec_of": (_I, [_I, _I, _I]),
+    "nvfp4_fp4_fallback": (_I, [_I]),
+    "nvfp4_node_exec": (_I, [_I, _I, _P, _P, _I, _P]),
     "nvfp4_set_fp4_kernel_disabled": (None, [_I]),
     "nvfp4_pair_name": (_S, [_I, _I]),
     "nvfp4_exec_name": (_S, [_I]),
@@ -145,6 +148,25 @@ def nvfp4_exec_of_arch(sm_arch: int, weight: Fmt, activation: Fmt,
                        fp4_kernel_disabled: bool = False) -> Exec:
     return Exec(load_library().nvfp4_exec_of_arch(int(sm_arch), int(weight), int(activation),
                                                   int(bool(fp4_kernel_disabled))))
+
+
+def nvfp4_fp4_fallback(sm_arch: int) -> Exec:
+    """How an NVFP4 activation runs on class sm_arch without an FP4 block-scale kernel."""
+    return Exec(load_library().nvfp4_fp4_fallback(int(sm_arch)))
+
+
+def nvfp4_node_exec(sm_arch: int, nodes, fp4_kernel_disabled: bool = False) -> list:
+    """node_exec over a list of (weight Fmt, activation Fmt) nodes on class sm_arch."""
+    import ctypes
+    nodes = list(nodes)
+    n = len(nodes)
+    w = (ctypes.c_int32 * max(n, 1))(*[int(a) for a, _ in nodes])
+    a = (ctypes.c_int32 * max(n, 1))(*[int(b) for _, b in nodes])
+    out = (ctypes.c_int32 * max(n, 1))()
+    _err(load_library().nvfp4_node_exec(int(sm_arch), int(bool(fp4_kernel_disabled)),
+                                        ctypes.cast(w, ctypes.c_void_p), ctypes.cast(a, ctypes.c_void_p),
+                                        n, ctypes.cast(out, ctypes.c_void_p)))
+    return [Exec(out[i]) for i in range(n)]
 
 
 def nvfp4_exec_of(device: int, weight: Fmt, activation: Fmt) -> Exec:

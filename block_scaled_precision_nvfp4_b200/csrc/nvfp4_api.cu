@@ -327,6 +327,19 @@ nvfp4_exec nvfp4_exec_of_arch(int arch, nvfp4_fmt weight, nvfp4_fmt activation,
     }
 }
 
+nvfp4_exec nvfp4_fp4_fallback(int sm_arch) { return fp4_fallback(sm_arch); }
+
+nvfp4_status nvfp4_node_exec(int sm_arch, int fp4_kernel_disabled, const int32_t* weight_fmt,
+                             const int32_t* activation_fmt, int n, int32_t* exec_out) {
+    if (n < 0) return fail(NVFP4_ERR_INVALID_ARG, "node count must be >= 0 (got %d)", n);
+    if (n > 0 && (!weight_fmt || !activation_fmt || !exec_out))
+        return fail(NVFP4_ERR_INVALID_ARG, "null node array");
+    for (int i = 0; i < n; ++i)
+        exec_out[i] = (int32_t)nvfp4_exec_of_arch(sm_arch, (nvfp4_fmt)weight_fmt[i],
+                                                  (nvfp4_fmt)activation_fmt[i], fp4_kernel_disabled);
+    return ok();
+}
+
 nvfp4_exec nvfp4_exec_of(int device, nvfp4_fmt weight, nvfp4_fmt activation) {
     DevInfo info;
     if (!device_info(device, info)) return NVFP4_EXEC_NO_PATH;

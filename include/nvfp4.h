@@ -110,6 +110,30 @@ NVFP4_API nvfp4_exec nvfp4_exec_of_arch(int sm_arch, nvfp4_fmt weight, nvfp4_fmt
  * the device cannot be queried).  Honors nvfp4_set_fp4_kernel_disabled(). */
 NVFP4_API nvfp4_exec nvfp4_exec_of(int device, nvfp4_fmt weight, nvfp4_fmt activation);
 
+/* fp4_fallback (metrale_circuit `hardware::exec`, fp4_fallback): how an NVFP4
+ * activation runs on class `sm_arch` when no FP4 block-scale kernel is
+ * compiled for it.  NO_FP4_KERNEL where the class has the FP4 MMA and only the
+ * kernel is missing (sm_100 with the switch below, sm_101/103/110/120/121);
+ * FP8_EXACT on a class without the FP4 MMA that has the FP8 MMA and this
+ * library's exact-path kernel (none besides sm_100, so in practice never);
+ * NO_PATH otherwise.  Pure function; usable without a GPU. */
+NVFP4_API nvfp4_exec nvfp4_fp4_fallback(int sm_arch);
+
+/* node_exec over a list of weight-reading nodes (metrale_circuit
+ * `hardware::exec`, node_exec): exec_out[i] is how node i, declared as
+ * (weight_fmt[i], activation_fmt[i]), runs on class `sm_arch`.  That is
+ * exec_of's answer, or fp4_fallback's where the class compiles no FP4
+ * block-scale kernel (fp4_kernel_disabled != 0 mimics such a class).  Format
+ * values outside nvfp4_fmt give NO_PATH for their node.  The arrays are host
+ * memory of n int32 each, read or written during the call only.  Returns
+ * NVFP4_ERR_INVALID_ARG for n < 0 or a null array with n > 0; n == 0 is OK.
+ * A declared format is never planned at a wider one: a node's answer is
+ * FP4_MMA only for NVFP4 activations, FP8_EXACT only for NVFP4 weights under
+ * NVFP4 or FP8 activations, BF16_WIDEN only for BF16 activations. */
+NVFP4_API nvfp4_status nvfp4_node_exec(int sm_arch, int fp4_kernel_disabled,
+                                       const int32_t* weight_fmt, const int32_t* activation_fmt,
+                                       int n, int32_t* exec_out);
+
 /* Process-wide switch that mimics a device class without a compiled FP4
  * block-scale kernel (for planning tests): while set, exec_of reports
  * NO_FP4_KERNEL for (NVFP4, NVFP4) and gemm_nvfp4_w4a4 / the grouped entry

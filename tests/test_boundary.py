@@ -173,3 +173,57 @@ def test_w4a8_argument_errors_need_no_device():
     assert call(A=0) == nv.Status.INVALID_ARG
     assert call(sW=40) == nv.Status.MISALIGNED
     assert call(Y=8) == nv.Status.MISALIGNED
+
+
+@pytest.mark.parametrize("arch,expect", [
+    (100, "NO_FP4_KERNEL"), (103, "NO_FP4_KERNEL"), (120, "NO_FP4_KERNEL"), (90, "NO_PATH"),
+    (89, "NO_PATH"), (80, "NO_PATH")])
+def test_fp4_fallback_by_class(arch, expect):
+    # a class with the FP4 MMA lacks only the kernel; other classes would need this
+    # library's exact-path kernel, which is compiled for sm_100 only
+    assert nv.nvfp4_fp4_fallback(arch).name == expect
+
+
+ALL_PAIRS = [(w, a) for w in nv.Fmt for a in nv.Fmt]
+
+
+@pytest.mark.parametrize("arch", [100, 103, 120, 90, 89, 80])
+@pytest.mark.parametrize("disabled", [False, True])
+def test_node_exec_is_exec_of_per_node(arch, disabled):
+    nodes = ALL_PAIRS * 2
+    got = nv.nvfp4_node_exec(arch, nodes, fp4_kernel_disabled=disabled)
+    assert got == [nv.nvfp4_exec_of_arch(arch, w, a, disabled) for w, a in nodes]
+
+
+def test_node_exec_without_fp4_kernel_takes_fp4_fallback():
+    F, E = nv.Fmt, nv.Exec
+    nodes = [(F.NVFP4, F.NVFP4), (F.NVFP4, F.FP8_E4M3), (F.NVFP4, F.BF16), (F.FP8_E4M3, F.FP8_E4M3)]
+    assert nv.nvfp4_node_exec(100, nodes) == [E.FP4_MMA, E.FP8_EXACT, E.BF16_WIDEN, E.NO_PATH]
+    assert nv.nvfp4_node_exec(100, nodes, fp4_kernel_disabled=True) == [
+        nv.nvfp4_fp4_fallback(100), E.FP8_EXACT, E.BF16_WIDEN, E.NO_PATH]
+
+
+def test_node_exec_never_plans_a_wider_format():
+    F, E = nv.Fmt, nv.Exec
+    for arch in (100, 101, 103, 110, 120, 121, 90, 89, 80, 75):
+        for disabled in (False, True):
+            for (w, a), e in zip(ALL_PAIRS, nv.nvfp4_node_exec(arch, ALL_PAIRS, disabled)):
+                if e == E.FP4_MMA:
+                    assert a == F.NVFP4 and w == F.NVFP4
+                if e == E.FP8_EXACT:
+                    assert w == F.NVFP4 and a in (F.NVFP4, F.FP8_E4M3)
+                if e == E.BF16_WIDEN:
+                    assert a == F.BF16
+
+
+def test_node_exec_bad_formats_and_arguments():
+    lib = nv.load_library()
+    w = (ctypes.c_int32 * 3)(2, 7, -1)
+    a = (ctypes.c_int32 * 3)(2, 2, 2)
+    out = (ctypes.c_int32 * 3)(-9, -9, -9)
+    assert lib.nvfp4_node_exec(100, 0, w, a, 3, out) == nv.Status.OK
+    assert list(out) == [nv.Exec.FP4_MMA, nv.Exec.NO_PATH, nv.Exec.NO_PATH]
+    assert lib.nvfp4_node_exec(100, 0, w, a, -1, out) == nv.Status.INVALID_ARG
+    assert lib.nvfp4_node_exec(100, 0, None, a, 3, out) == nv.Status.INVALID_ARG
+    assert lib.nvfp4_node_exec(100, 0, None, None, 0, None) == nv.Status.OK
+    assert nv.nvfp4_node_exec(100, []) == []
