@@ -649,13 +649,15 @@ nvfp4_status gemm_nvfp4_w4a8(const uint8_t* A_fp8, float gA, const uint8_t* W, c
 
     nvfp4_status st;
     CUtensorMap tmA, tmB, tmSB;
-    if ((st = make_map_u8(&tmA, A_fp8, (uint64_t)K, (uint64_t)M, 128, k8::BM)) != NVFP4_OK) return st;
-    if ((st = make_map_u8(&tmB, W, (uint64_t)K / 2, (uint64_t)N, 128, k8::BN)) != NVFP4_OK) return st;
-    if ((st = make_map_u8(&tmSB, sW, (uint64_t)K / 16, (uint64_t)N, 16, k8::BN,
+    // activations: 128-byte-wide boxes of the tile's 256 token rows (the MMA's B side);
+    // weights: 128-byte boxes of the tile's 128 weight rows (converted into TMEM)
+    if ((st = make_map_u8(&tmA, A_fp8, (uint64_t)K, (uint64_t)M, 128, k8::BT)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmB, W, (uint64_t)K / 2, (uint64_t)N, 128, k8::BW)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmSB, sW, (uint64_t)K / 16, (uint64_t)N, 16, k8::BW,
                           CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
         return st;
     if ((st = set_smem(k8::w4a8_kernel, k8::SMEM_BYTES, info, "w4a8_kernel")) != NVFP4_OK) return st;
-    const int tiles = ((M + k8::BM - 1) / k8::BM) * ((N + k8::BN - 1) / k8::BN);
+    const int tiles = ((M + k8::BT - 1) / k8::BT) * ((N + k8::BW - 1) / k8::BW);
     const int grid = tiles < info.num_sms ? tiles : info.num_sms;
     k8::w4a8_kernel<<<grid, k8::NUM_THREADS, k8::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
         tmA, tmB, tmSB, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K, gA * gW);

@@ -1,39 +1,42 @@
-// w4a8_kernel.cuh -- FP8 (E4M3) activations under NVFP4 weights on the exact
-// E4M3 path (metrale_circuit `hardware::exec`, exec_of: "NVFP4 weights under
-// FP8 activations (W4A8 with group-16 E4M3 scales) have no single-instruction
-// MMA ...; they take the exact E4M3 path").
+// w4a8_kernel.cuh -- FP8 (E4M3) activations under NVFP4 weights on the FP8
+// tensor-core MMA, exactly (metrale_circuit `hardware::exec`, exec_of: W4A8
+// with group-16 E4M3 weight scales has no single-instruction MMA and takes the
+// exact E4M3 path):
 //
 //     Y[m,n] = gA*gW * sum_g sW[n,g] * sum_{k in g} a8[m,k] * e2m1(W[n,k])
 //
-// The weights go through the page's identity (each code in the high nibble of
-// a byte: (q & 0x80808080) | ((q & 0x70707070) >> 2), an E4M3 byte worth the
-// code's value times 2^-6); the activations are E4M3 already.  For every
-// 16-group an FP8 MMA (kind::f8f6f4, E4M3 x E4M3 -> FP32, K = 32) forms the
-// group's partial, and the weights' group scale with the folded 2^6 is applied
-// in FP32 per K = 16 step:  acc[m,n] += P_g[m,n] * (sW[n,g] * 2^6).
-// Each product has at most 6 significant bits, so P_g is exact in FP32 unless
-// the group's nonzero products span more than 2^15 in magnitude; the scale
-// apply is one fused multiply-add.
+// The activations go to the FP8 MMA as they are.  The weights go through an
+// exact conversion that carries the group scale inside the operand, so the
+// FP32 accumulator stays in tensor memory for the whole of K (no per-group
+// partial leaves TMEM):
 //
-// One K = 32 MMA covers one group: A's K = 32 slice (two groups) comes straight
-// from the TMA-loaded, 128-byte-swizzled activation tile, and B holds the group
-// in one 16-byte K chunk and a shared all-zero tile in the other (reached
-// through the smem descriptor's leading byte offset), so the other group of
-// the slice contributes nothing.
+//  * a scale byte s is x * 2^b with x an integer in 0..15 (x = 8 + mantissa,
+//    b = E - 10 for a normal byte; x = mantissa, b = -9 for a subnormal one);
+//  * x is written in non-adjacent form, x = sum_i sigma_i * 2^t_i with at most
+//    three nonzero signed digits (x3 = x + (x >> 1), c = (x >> 1) ^ x3: the
+//    positive digits are x3 & c, the negative ones (x >> 1) & c);
+//  * plane i of a weight is sigma_i * e2m1(w) * 2^(t_i + b), an E5M2 byte: an
+//    E2M1 value has two significant bits, and |t_i + b| <= 9 keeps every value
+//    inside E5M2's normal range, so the byte is exact;
+//  * sum_i plane_i = e2m1(w) * s, so three E4M3 x E5M2 MMAs per K step, one per
+//    plane, accumulate sum_k a8 * w * s in FP32 exactly as the declared W4A4
+//    block-scaled product would (each product exact, FP32 accumulation).
 //
-// Roles (one persistent CTA per SM, 12 warps, 128 x 128 output tiles), as on
-// the W4A4 exact path (via_fp8_kernel.cuh):
-//   warp 0      TMA producer: E4M3 activation K-blocks (256 bytes of a row as
-//               two 128-byte swizzled boxes), packed FP4 weight K-blocks and
-//               the weights' raw [rows][16 B] scale tiles.
-//   warp 1      TMEM owner, MMA issuer: one MMA per group into a 4-deep ring of
-//               128-column FP32 partial buffers; it also releases the raw stage
-//               (its MMAs read the activations there).
-//   warps 2-3   converters: weight codes -> E4M3 per-group [rows][16 B] tiles;
-//               weight scales -> FP32 (x 2^6).
-//   warps 4-11  scale-apply + epilogue: per group, partial TMEM -> registers,
-//               acc += P * (sW*64) with packed f32x2 FMAs; at the end of a
-//               tile, x alpha, BF16 RNE, store.
+// Operand placement: the weight planes are the MMA's A operand (M = 128 weight
+// rows) and live in tensor memory, written there by the converter warps with
+// tcgen05.st straight from registers; the activations are the B operand
+// (N = 256 tokens), 128-byte-swizzled tiles loaded by TMA.  The accumulator is
+// D[weight row][token]; the epilogue writes Y[token][weight row].
+//
+// Roles (one persistent CTA per SM, 10 warps, tiles of 128 weight rows x 256
+// tokens):
+//   warp 0      TMA producer: activation K-blocks (two 128-byte boxes of 256
+//               rows), packed weight K-blocks and their raw scale tiles.
+//   warp 1      TMEM owner (512 columns: accumulator 256, plane ring 8 x 24),
+//               MMA issuer.
+//   warps 2-5   converters, one weight row per thread (TMEM lane): per K step,
+//               32 codes -> three planes of 32 E5M2 bytes -> tcgen05.st.
+//   warps 6-9   epilogue: TMEM -> registers, x alpha, BF16 RNE, store.
 // Requires K % 256 == 0 (TMA of the scale tiles).
 #pragma once
 #include <cuda_bf16.h>
@@ -45,43 +48,121 @@
 namespace nvfp4 {
 namespace w4a8 {
 
-using via_fp8::convert8;
-using via_fp8::fma2;
-using via_fp8::pack2;
-using via_fp8::scale_x64;
 using via_fp8::tile_coords;
 using via_fp8::warp_wait;
 
-constexpr int BM = 128, BN = 128;
-constexpr int BK = 256;              // codes per raw K-block (16 groups)
-constexpr int RSTAGES = 3;           // raw K-block ring
-constexpr int NSLOTS = 4;            // converted group-pair ring
-constexpr int NPART = 4;             // TMEM partial buffers (128 columns each)
-constexpr int CONV_WARPS = 2, APPLY_WARPS = 8;
-constexpr int NUM_THREADS = 32 * (2 + CONV_WARPS + APPLY_WARPS);
+constexpr int BW = 128;               // weight rows per tile (TMEM lanes, the MMA's M)
+constexpr int BT = 256;               // tokens per tile (the MMA's N)
+constexpr int BK = 256;               // codes per raw K-block
+constexpr int STEPS = BK / 32;        // K = 32 MMA steps per K-block
+constexpr int RSTAGES = 2;            // raw K-block ring
+constexpr int PLANES = 3;             // signed digits of a scale, at most
+constexpr int NSLOT = 8;              // TMEM plane-slot ring, one K step each
+constexpr int SLOT_COLS = PLANES * 8; // 32 bytes of K per lane = 8 columns per plane
+constexpr int ACC_COLS = BT;          // FP32 accumulator columns
+constexpr int TMEM_COLS = 512;
+constexpr int CONV_WARPS = 4, EPI_WARPS = 4;
+constexpr int NUM_THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
+static_assert(ACC_COLS + NSLOT * SLOT_COLS <= TMEM_COLS, "TMEM budget");
 
-enum Role { ROLE_PRODUCER = 1, ROLE_MMA = 2, ROLE_CONV = 3, ROLE_APPLY = 4, ROLE_DRAIN = 5 };
+enum Role { ROLE_PRODUCER = 1, ROLE_MMA = 2, ROLE_CONV = 3, ROLE_EPI = 4, ROLE_DRAIN = 5 };
 
 struct Smem {
-    alignas(1024) uint8_t raw_a[RSTAGES][2][BM * 128];  // E4M3 activations, two swizzled boxes
-    alignas(1024) uint8_t raw_b[RSTAGES][BN * 128];     // packed FP4 weights, swizzled
-    alignas(16) uint8_t raw_sb[RSTAGES][BN * 16];       // weight scales [row][16 groups]
-    alignas(128) uint8_t zlo[BN * 16];                  // zero tile below every b8 tile
-    alignas(128) uint8_t b8[NSLOTS][2][BN * 16];        // [slot][group of pair][row][16 B]
-    alignas(128) uint8_t zhi[BN * 16];                  // zero tile above every b8 tile
-    alignas(16) float sw_f[NSLOTS][2][BN];              // sW * 2^6
+    alignas(1024) uint8_t act[RSTAGES][2][BT * 128];  // E4M3 activations, two swizzled boxes
+    alignas(1024) uint8_t w[RSTAGES][BW * 128];       // packed FP4 weights, swizzled
+    alignas(16) uint8_t sw[RSTAGES][BW * 16];         // weight scales [row][16 groups]
     uint64_t raw_full[RSTAGES], raw_empty[RSTAGES];
-    uint64_t slot_full[NSLOTS], slot_empty[NSLOTS];
-    uint64_t part_full[NPART], part_empty[NPART];
+    uint64_t slot_full[NSLOT], slot_empty[NSLOT];
+    uint64_t acc_full, acc_empty;
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
 constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
-constexpr uint32_t RAW_BYTES = BM * 256 + BN * 128 + BN * 16;
+constexpr uint32_t RAW_BYTES = BT * 256 + BW * 128 + BW * 16;
+
+// kind::f8f6f4 instruction descriptor: F32 accumulator, A and B formats
+// (0 = E4M3, 1 = E5M2), both K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_f8f6f4(uint32_t M, uint32_t N, uint32_t afmt,
+                                                    uint32_t bfmt) {
+    return (1u << 4) | (afmt << 7) | (bfmt << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// D (TMEM) += A (TMEM, K-major: row i in lane i, K bytes along the columns) x B (smem).
+__device__ __forceinline__ void mma_f8f6f4_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// This warp's 32 lanes x 8 consecutive 32-bit columns from registers.
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// One plane of one group: an 8-entry byte table T[c] = E5M2(e2m1(c) * 2^p) for
+// the magnitude codes c = 0..7 (T[0] = 0), as two words for byte_perm, and the
+// digit's sign as a byte mask.  With base = (p + 14) << 2 the E5M2 bytes are
+//   c=1 (0.5): base         c=2 (1): base + 4    c=3 (1.5): base + 6
+//   c=4 (2):   base + 8     c=5 (3): base + 10   c=6 (4):   base + 12
+//   c=7 (6):   base + 14
+// (exponent field p + 14 + e2m1 exponent, mantissa bit of the code in bit 1).
+struct PlaneTable {
+    uint32_t lo, hi, sgn;
+};
+
+__device__ __forceinline__ void plane_tables(uint32_t sb, PlaneTable (&t)[PLANES]) {
+    const uint32_t E = (sb >> 3) & 15u, mt = sb & 7u;
+    const uint32_t x = E ? (8u | mt) : mt;
+    const int b = E ? (int)E - 10 : -9;
+    const uint32_t xh = x >> 1, x3 = x + xh, c = xh ^ x3;
+    const uint32_t neg = xh & c;
+    uint32_t d = (x3 & c) | neg;  // digit positions, at most three
+#pragma unroll
+    for (int i = 0; i < PLANES; ++i) {
+        if (d) {
+            const int ti = __ffs(d) - 1;
+            d &= d - 1;
+            const uint32_t base = (uint32_t)(ti + b + 14) << 2;
+            t[i].lo = base * 0x01010100u + 0x06040000u;
+            t[i].hi = base * 0x01010101u + 0x0E0C0A08u;
+            t[i].sgn = ((neg >> ti) & 1u) ? 0x80808080u : 0u;
+        } else {
+            t[i].lo = 0u;
+            t[i].hi = 0u;
+            t[i].sgn = 0u;
+        }
+    }
+}
+
+// Eight packed codes (code j in nibble j) -> for each plane, two words of E5M2
+// bytes in k order (byte j of the first word = code j).
+__device__ __forceinline__ void convert8_planes(uint32_t w, const PlaneTable (&t)[PLANES],
+                                                uint32_t (&out)[PLANES][2]) {
+    const uint32_t sel_lo = w & 0x7777u, sel_hi = (w >> 16) & 0x7777u;
+    // 0x80 in byte j where code j is negative: byte_perm of (byte 0 = 0, byte 1 = 0x80)
+    const uint32_t sg_lo = __byte_perm(0x8000u, 0u, (w >> 3) & 0x1111u);
+    const uint32_t sg_hi = __byte_perm(0x8000u, 0u, (w >> 19) & 0x1111u);
+#pragma unroll
+    for (int i = 0; i < PLANES; ++i) {
+        out[i][0] = __byte_perm(t[i].lo, t[i].hi, sel_lo) | (sg_lo ^ t[i].sgn);
+        out[i][1] = __byte_perm(t[i].lo, t[i].hi, sel_hi) | (sg_hi ^ t[i].sgn);
+    }
+}
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B x 128 rows
+w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B x 256 rows
             const __grid_constant__ CUtensorMap tmB,   // packed W [N][K/2], box 128 B x 128 rows
             const __grid_constant__ CUtensorMap tmSB,  // sW [N][K/16], box 16 B x 128 rows
             __nv_bfloat16* __restrict__ Y, int M, int N, int K, float alpha) {
@@ -89,8 +170,8 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
-    const int tiles = num_m * num_n;
+    const int num_t = (M + BT - 1) / BT, num_w = (N + BW - 1) / BW;
+    const int tiles = num_t * num_w;
     const int num_kb = K / BK;
     volatile int* abort = &sm.abort;
 
@@ -99,14 +180,12 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
             mbar_init(&sm.raw_full[s], 1);
             mbar_init(&sm.raw_empty[s], CONV_WARPS + 1);  // converters + the MMA's commit
         }
-        for (int s = 0; s < NSLOTS; ++s) {
+        for (int s = 0; s < NSLOT; ++s) {
             mbar_init(&sm.slot_full[s], CONV_WARPS);
-            mbar_init(&sm.slot_empty[s], 1 + APPLY_WARPS);
+            mbar_init(&sm.slot_empty[s], 1);
         }
-        for (int p = 0; p < NPART; ++p) {
-            mbar_init(&sm.part_full[p], 1);
-            mbar_init(&sm.part_empty[p], APPLY_WARPS);
-        }
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.acc_empty, EPI_WARPS);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbarrier_init();
@@ -114,13 +193,8 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmSB);
     }
-    for (int i = threadIdx.x; i < BN * 16 / 4; i += NUM_THREADS) {
-        reinterpret_cast<uint32_t*>(sm.zlo)[i] = 0u;
-        reinterpret_cast<uint32_t*>(sm.zhi)[i] = 0u;
-    }
-    fence_proxy_async_smem();
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, NPART * 128);
+        tmem_alloc(&sm.tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -133,17 +207,17 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
         if (lane == 0) {
             int it = 0;
             for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
-                int mb, nb;
-                tile_coords(tile, num_m, num_n, mb, nb);
+                int tt, tw;
+                tile_coords(tile, num_t, num_w, tt, tw);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int r = it % RSTAGES;
                     if (!mbar_wait(&sm.raw_empty[r], ((it / RSTAGES) & 1) ^ 1, abort, ROLE_PRODUCER))
                         goto producer_done;
                     mbar_arrive_expect_tx(&sm.raw_full[r], RAW_BYTES);
-                    tma_load_2d(sm.raw_a[r][0], &tmA, &sm.raw_full[r], kb * 256, mb * BM);
-                    tma_load_2d(sm.raw_a[r][1], &tmA, &sm.raw_full[r], kb * 256 + 128, mb * BM);
-                    tma_load_2d(sm.raw_b[r], &tmB, &sm.raw_full[r], kb * 128, nb * BN);
-                    tma_load_2d(sm.raw_sb[r], &tmSB, &sm.raw_full[r], kb * 16, nb * BN);
+                    tma_load_2d(sm.act[r][0], &tmA, &sm.raw_full[r], kb * 256, tt * BT);
+                    tma_load_2d(sm.act[r][1], &tmA, &sm.raw_full[r], kb * 256 + 128, tt * BT);
+                    tma_load_2d(sm.w[r], &tmB, &sm.raw_full[r], kb * 128, tw * BW);
+                    tma_load_2d(sm.sw[r], &tmSB, &sm.raw_full[r], kb * 16, tw * BW);
                 }
             }
         producer_done:
@@ -159,40 +233,32 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_f8f6f4_e4m3(BM, BN);
-            const uint32_t zlo = smem_u32(sm.zlo), zhi = smem_u32(sm.zhi);
-            int pc = 0, gc = 0, it = 0;
+            const uint32_t idesc = idesc_f8f6f4(BW, BT, /*A E5M2*/ 1u, /*B E4M3*/ 0u);
+            int it = 0, st = 0, tc = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
+                // the epilogue has read the previous tile's accumulator
+                if (!mbar_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
+                tc_fence_after();
                 for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
                     const int r = it % RSTAGES;
-                    // the activations are read from the raw stage itself: wait for its
-                    // TMA bytes here too (the stage cannot be refilled before this
-                    // K-block's commit below, so the phase cannot run ahead)
                     if (!mbar_wait(&sm.raw_full[r], (it / RSTAGES) & 1, abort, ROLE_MMA)) { ok = false; break; }
-                    for (int h = 0; h < 8 && ok; ++h, ++pc) {
-                        const int sl = pc % NSLOTS;
-                        if (!mbar_wait(&sm.slot_full[sl], (pc / NSLOTS) & 1, abort, ROLE_MMA)) { ok = false; break; }
-                        // A: the pair's 32 bytes of the row (groups 2h, 2h+1), straight from
-                        // the swizzled activation box
-                        const uint64_t adesc =
-                            desc_kmajor_sw128(smem_u32(sm.raw_a[r][h >> 2]) + (h & 3) * 32);
-                        const uint32_t b0 = smem_u32(sm.b8[sl][0]), b1 = smem_u32(sm.b8[sl][1]);
+                    for (int h = 0; h < STEPS; ++h, ++st) {
+                        const int s = st % NSLOT;
+                        if (!mbar_wait(&sm.slot_full[s], (st / NSLOT) & 1, abort, ROLE_MMA)) { ok = false; break; }
+                        tc_fence_after();
+                        // B: the K = 32 slice of the 256 activation rows (128-byte swizzle)
+                        const uint64_t bdesc =
+                            desc_kmajor_sw128(smem_u32(sm.act[r][h >> 2]) + (h & 3) * 32);
+                        const uint32_t a0 = tmem + ACC_COLS + s * SLOT_COLS;
 #pragma unroll
-                        for (int gi = 0; gi < 2; ++gi, ++gc) {
-                            const int p = gc % NPART;
-                            if (!mbar_wait(&sm.part_empty[p], ((gc / NPART) & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
-                            tc_fence_after();
-                            // B: the group in its own K chunk, the other chunk all zero
-                            const uint64_t bdesc = gi == 0 ? smem_desc(b0, zhi - b0, 128, 0)
-                                                           : smem_desc(zlo, b1 - zlo, 128, 0);
-                            mma_f8f6f4(tmem + p * 128, adesc, bdesc, idesc, 0u);
-                            mma_commit(&sm.part_full[p]);
-                        }
-                        if (ok) mma_commit(&sm.slot_empty[sl]);
+                        for (int i = 0; i < PLANES; ++i)
+                            mma_f8f6f4_ts(tmem, a0 + i * 8, bdesc, idesc, (kb | h | i) != 0);
+                        mma_commit(&sm.slot_empty[s]);
                     }
                     if (ok) mma_commit(&sm.raw_empty[r]);  // the activations of this stage are read
                 }
+                if (ok) mma_commit(&sm.acc_full);
             }
             mma_commit(&sm.drain);
             const uint64_t t0 = globaltimer_ns();
@@ -204,120 +270,81 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
             }
         }
     } else if (warp < 2 + CONV_WARPS) {
-        // ------------------------------------------------------------ converters (weights)
-        const int ctid = threadIdx.x - 64;  // 0..63: weight rows ctid and ctid + 64
-        int it = 0, pc = 0;
+        // ------------------------------------------------------------ converters
+        const int q = warp & 3;            // TMEM lane quarter this warp may access
+        const int row = 32 * q + lane;     // weight row within the tile
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + ACC_COLS;
+        int it = 0, st = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
                 const int r = it % RSTAGES;
                 if (!warp_wait(&sm.raw_full[r], (it / RSTAGES) & 1, abort, ROLE_CONV)) { ok = false; break; }
-                uint32_t sbw[2][4];
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const uint4 b = *reinterpret_cast<const uint4*>(sm.raw_sb[r] + (ctid + 64 * rr) * 16);
-                    sbw[rr][0] = b.x; sbw[rr][1] = b.y; sbw[rr][2] = b.z; sbw[rr][3] = b.w;
-                }
+                const uint4 sbq = *reinterpret_cast<const uint4*>(sm.sw[r] + row * 16);
+                const uint32_t sbw[4] = {sbq.x, sbq.y, sbq.z, sbq.w};
 #pragma unroll 1
-                for (int h = 0; h < 8; ++h, ++pc) {
-                    const int sl = pc % NSLOTS;
-                    if (!warp_wait(&sm.slot_empty[sl], ((pc / NSLOTS) & 1) ^ 1, abort, ROLE_CONV)) { ok = false; break; }
-                    const int g0 = 2 * h, g1 = 2 * h + 1;
+                for (int h = 0; h < STEPS; ++h, ++st) {
+                    const int s = st % NSLOT;
+                    // K step h: codes 32h .. 32h+31 of the row (16 bytes, chunk h of the
+                    // 128-byte swizzled row), groups 2h and 2h+1
+                    const uint4 qb = *reinterpret_cast<const uint4*>(
+                        sm.w[r] + row * 128 + ((h ^ (row & 7)) << 4));
+                    PlaneTable t0[PLANES], t1[PLANES];
+                    plane_tables((sbw[h >> 1] >> (16 * (h & 1))) & 0xFFu, t0);
+                    plane_tables((sbw[h >> 1] >> (16 * (h & 1) + 8)) & 0xFFu, t1);
+                    uint32_t o0[PLANES][2], o1[PLANES][2], o2[PLANES][2], o3[PLANES][2];
+                    convert8_planes(qb.x, t0, o0);
+                    convert8_planes(qb.y, t0, o1);
+                    convert8_planes(qb.z, t1, o2);
+                    convert8_planes(qb.w, t1, o3);
+                    if (!warp_wait(&sm.slot_empty[s], ((st / NSLOT) & 1) ^ 1, abort, ROLE_CONV)) { ok = false; break; }
+                    tc_fence_after();
 #pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int row = ctid + 64 * rr;
-                        // 16-byte chunk h of the row (groups 2h, 2h+1) under the 128-byte swizzle
-                        const uint4 qb = *reinterpret_cast<const uint4*>(
-                            sm.raw_b[r] + row * 128 + ((h ^ (row & 7)) << 4));
-                        const uint2 b0 = convert8(qb.x), b1 = convert8(qb.y), b2 = convert8(qb.z),
-                                    b3 = convert8(qb.w);
-                        *reinterpret_cast<uint4*>(sm.b8[sl][0] + row * 16) = make_uint4(b0.x, b0.y, b1.x, b1.y);
-                        *reinterpret_cast<uint4*>(sm.b8[sl][1] + row * 16) = make_uint4(b2.x, b2.y, b3.x, b3.y);
-                        sm.sw_f[sl][0][row] = scale_x64((sbw[rr][g0 >> 2] >> (8 * (g0 & 3))) & 0xFFu);
-                        sm.sw_f[sl][1][row] = scale_x64((sbw[rr][g1 >> 2] >> (8 * (g1 & 3))) & 0xFFu);
+                    for (int i = 0; i < PLANES; ++i) {
+                        const uint32_t v[8] = {o0[i][0], o0[i][1], o1[i][0], o1[i][1],
+                                               o2[i][0], o2[i][1], o3[i][0], o3[i][1]};
+                        tmem_st_32x32b_x8(tq + s * SLOT_COLS + i * 8, v);
                     }
-                    fence_proxy_async_smem();
+                    tmem_st_wait();
+                    tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.slot_full[sl]);
+                    if (lane == 0) mbar_arrive(&sm.slot_full[s]);
                 }
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(&sm.raw_empty[r]);
             }
         }
     } else {
-        // ------------------------------------------------------------ scale-apply + epilogue
-        const int q = warp & 3;                         // TMEM lane quarter
-        const int half = (warp - 2 - CONV_WARPS) >> 2;  // column half
-        const int trow = 32 * q + lane;                 // row within the tile
-        const bool vec_ok = (N % 8) == 0;
-        int pc = 0, gc = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-            int mb, nb;
-            tile_coords(tile, num_m, num_n, mb, nb);
-            uint64_t acc[32];
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+        int tc = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tc) {
+            int tt, tw;
+            tile_coords(tile, num_t, num_w, tt, tw);
+            if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI)) break;
+            tc_fence_after();
+            const int n = tw * BW + 32 * q + lane;   // this thread's weight row = output column
+            const int m0 = tt * BT;
+#pragma unroll 1
+            for (int c = 0; c < BT / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tq + 32 * c, v);
+                tmem_ld_wait();
+                reg_fence(v);
+                if (c == BT / 32 - 1) {  // the whole accumulator is read: release it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.acc_empty);
+                }
+                if (n < N) {
+                    // token m0 + 32c + j; the warp's 32 lanes write 64 contiguous bytes
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] = 0ull;
-            for (int pair = 0; pair < num_kb * 8 && ok; ++pair, ++pc) {
-                const int sl = pc % NSLOTS;
-                if (!warp_wait(&sm.slot_full[sl], (pc / NSLOTS) & 1, abort, ROLE_APPLY)) { ok = false; break; }
-#pragma unroll
-                for (int gi = 0; gi < 2; ++gi, ++gc) {
-                    const int p = gc % NPART;
-                    if (!warp_wait(&sm.part_full[p], (gc / NPART) & 1, abort, ROLE_APPLY)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + p * 128 + half * 64;
-                    const float4* sw4 = reinterpret_cast<const float4*>(&sm.sw_f[sl][gi][half * 64]);
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(ta + 32 * c, v);
-                        tmem_ld_wait();
-                        reg_fence(v);
-                        if (c == 1) {  // the whole partial is in registers: release it
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&sm.part_empty[p]);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 w4 = sw4[8 * c + j];
-                            acc[16 * c + 2 * j] = fma2(pack2(v[4 * j], v[4 * j + 1]),
-                                                       pack2(__float_as_uint(w4.x), __float_as_uint(w4.y)),
-                                                       acc[16 * c + 2 * j]);
-                            acc[16 * c + 2 * j + 1] = fma2(pack2(v[4 * j + 2], v[4 * j + 3]),
-                                                           pack2(__float_as_uint(w4.z), __float_as_uint(w4.w)),
-                                                           acc[16 * c + 2 * j + 1]);
-                        }
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + 32 * c + j;
+                        if (m < M)
+                            Y[(size_t)m * N + n] = __float2bfloat16_rn(__uint_as_float(v[j]) * alpha);
                     }
-                }
-                __syncwarp();
-                if (ok && lane == 0) mbar_arrive(&sm.slot_empty[sl]);
-            }
-            if (!ok) break;
-            // epilogue: x alpha, BF16 RNE, store this thread's 64 columns
-            const int row = mb * BM + trow;
-            const int col0 = nb * BN + half * 64;
-            if (row < M) {
-                uint32_t packed[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float lo = __uint_as_float((uint32_t)acc[j]) * alpha;
-                    const float hi = __uint_as_float((uint32_t)(acc[j] >> 32)) * alpha;
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
-                    packed[j] = *reinterpret_cast<uint32_t*>(&h2);
-                }
-                __nv_bfloat16* yrow = Y + (size_t)row * N;
-                if (vec_ok && col0 + 64 <= N) {
-                    uint4* dst = reinterpret_cast<uint4*>(yrow + col0);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-                } else {
-                    uint16_t* y16 = reinterpret_cast<uint16_t*>(yrow);
-#pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        if (col0 + j < N) y16[col0 + j] = (uint16_t)(packed[j >> 1] >> (16 * (j & 1)));
                 }
             }
         }
@@ -326,7 +353,7 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, NPART * 128);
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 }  // namespace w4a8
