@@ -28,15 +28,18 @@
 // (N = 256 tokens), 128-byte-swizzled tiles loaded by TMA.  The accumulator is
 // D[weight row][token]; the epilogue writes Y[token][weight row].
 //
-// Roles (one persistent CTA per SM, 10 warps, tiles of 128 weight rows x 256
+// Roles (one persistent CTA per SM, 14 warps, tiles of 128 weight rows x 256
 // tokens):
 //   warp 0      TMA producer: activation K-blocks (two 128-byte boxes of 256
 //               rows), packed weight K-blocks and their raw scale tiles.
 //   warp 1      TMEM owner (512 columns: accumulator 256, plane ring 8 x 24),
 //               MMA issuer.
-//   warps 2-5   converters, one weight row per thread (TMEM lane): per K step,
-//               32 codes -> three planes of 32 E5M2 bytes -> tcgen05.st.
-//   warps 6-9   epilogue: TMEM -> registers, x alpha, BF16 RNE, store.
+//   warps 2-9   converters, one weight row per thread (TMEM lane), two warps
+//               per lane quarter taking the even and the odd K steps: per step,
+//               32 codes -> three planes of 32 E5M2 bytes -> tcgen05.st.  The
+//               plane tables of every scale byte are built once per CTA in
+//               shared memory.
+//   warps 10-13 epilogue: TMEM -> registers, x alpha, BF16 RNE, store.
 // Requires K % 256 == 0 (TMA of the scale tiles).
 #pragma once
 #include <cuda_bf16.h>
@@ -61,9 +64,10 @@ constexpr int NSLOT = 8;              // TMEM plane-slot ring, one K step each
 constexpr int SLOT_COLS = PLANES * 8; // 32 bytes of K per lane = 8 columns per plane
 constexpr int ACC_COLS = BT;          // FP32 accumulator columns
 constexpr int TMEM_COLS = 512;
-constexpr int CONV_WARPS = 4, EPI_WARPS = 4;
+constexpr int CONV_WARPS = 8, EPI_WARPS = 4;  // two converter warps per TMEM lane quarter
 constexpr int NUM_THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
 static_assert(ACC_COLS + NSLOT * SLOT_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(NSLOT == STEPS, "one TMEM slot per K step of a block");
 
 enum Role { ROLE_PRODUCER = 1, ROLE_MMA = 2, ROLE_CONV = 3, ROLE_EPI = 4, ROLE_DRAIN = 5 };
 
@@ -71,6 +75,7 @@ struct Smem {
     alignas(1024) uint8_t act[RSTAGES][2][BT * 128];  // E4M3 activations, two swizzled boxes
     alignas(1024) uint8_t w[RSTAGES][BW * 128];       // packed FP4 weights, swizzled
     alignas(16) uint8_t sw[RSTAGES][BW * 16];         // weight scales [row][16 groups]
+    uint4 ptab[128][PLANES];                          // plane tables per scale byte (lo, hi, sgn)
     uint64_t raw_full[RSTAGES], raw_empty[RSTAGES];
     uint64_t slot_full[NSLOT], slot_empty[NSLOT];
     uint64_t acc_full, acc_empty;
@@ -181,7 +186,7 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
             mbar_init(&sm.raw_empty[s], CONV_WARPS + 1);  // converters + the MMA's commit
         }
         for (int s = 0; s < NSLOT; ++s) {
-            mbar_init(&sm.slot_full[s], CONV_WARPS);
+            mbar_init(&sm.slot_full[s], CONV_WARPS / 2);  // the four warps of the step's parity
             mbar_init(&sm.slot_empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
@@ -192,6 +197,12 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmSB);
+    }
+    if (threadIdx.x < 128) {  // the plane tables of scale byte threadIdx.x
+        PlaneTable t[PLANES];
+        plane_tables(threadIdx.x, t);
+#pragma unroll
+        for (int i = 0; i < PLANES; ++i) sm.ptab[threadIdx.x][i] = make_uint4(t[i].lo, t[i].hi, t[i].sgn, 0u);
     }
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, TMEM_COLS);
@@ -271,10 +282,11 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
         }
     } else if (warp < 2 + CONV_WARPS) {
         // ------------------------------------------------------------ converters
-        const int q = warp & 3;            // TMEM lane quarter this warp may access
-        const int row = 32 * q + lane;     // weight row within the tile
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int par = (warp - 2) >> 2;        // this warp's K steps: h = par, par + 2, ...
+        const int row = 32 * q + lane;          // weight row within the tile
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + ACC_COLS;
-        int it = 0, st = 0;
+        int it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
@@ -283,32 +295,38 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
                 const uint4 sbq = *reinterpret_cast<const uint4*>(sm.sw[r] + row * 16);
                 const uint32_t sbw[4] = {sbq.x, sbq.y, sbq.z, sbq.w};
 #pragma unroll 1
-                for (int h = 0; h < STEPS; ++h, ++st) {
-                    const int s = st % NSLOT;
-                    // K step h: codes 32h .. 32h+31 of the row (16 bytes, chunk h of the
-                    // 128-byte swizzled row), groups 2h and 2h+1
+                for (int h = par; h < STEPS; h += 2) {
+                    // K step h of the block uses TMEM slot h (STEPS == NSLOT)
+                    // codes 32h .. 32h+31 of the row: 16 bytes, chunk h of the 128-byte
+                    // swizzled row; groups 2h and 2h+1
                     const uint4 qb = *reinterpret_cast<const uint4*>(
                         sm.w[r] + row * 128 + ((h ^ (row & 7)) << 4));
+                    const uint32_t sb0 = (sbw[h >> 1] >> (16 * (h & 1))) & 0x7Fu;
+                    const uint32_t sb1 = (sbw[h >> 1] >> (16 * (h & 1) + 8)) & 0x7Fu;
                     PlaneTable t0[PLANES], t1[PLANES];
-                    plane_tables((sbw[h >> 1] >> (16 * (h & 1))) & 0xFFu, t0);
-                    plane_tables((sbw[h >> 1] >> (16 * (h & 1) + 8)) & 0xFFu, t1);
+#pragma unroll
+                    for (int i = 0; i < PLANES; ++i) {
+                        const uint4 a = sm.ptab[sb0][i], b = sm.ptab[sb1][i];
+                        t0[i].lo = a.x; t0[i].hi = a.y; t0[i].sgn = a.z;
+                        t1[i].lo = b.x; t1[i].hi = b.y; t1[i].sgn = b.z;
+                    }
                     uint32_t o0[PLANES][2], o1[PLANES][2], o2[PLANES][2], o3[PLANES][2];
                     convert8_planes(qb.x, t0, o0);
                     convert8_planes(qb.y, t0, o1);
                     convert8_planes(qb.z, t1, o2);
                     convert8_planes(qb.w, t1, o3);
-                    if (!warp_wait(&sm.slot_empty[s], ((st / NSLOT) & 1) ^ 1, abort, ROLE_CONV)) { ok = false; break; }
+                    if (!warp_wait(&sm.slot_empty[h], (it & 1) ^ 1, abort, ROLE_CONV)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int i = 0; i < PLANES; ++i) {
                         const uint32_t v[8] = {o0[i][0], o0[i][1], o1[i][0], o1[i][1],
                                                o2[i][0], o2[i][1], o3[i][0], o3[i][1]};
-                        tmem_st_32x32b_x8(tq + s * SLOT_COLS + i * 8, v);
+                        tmem_st_32x32b_x8(tq + h * SLOT_COLS + i * 8, v);
                     }
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.slot_full[s]);
+                    if (lane == 0) mbar_arrive(&sm.slot_full[h]);
                 }
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(&sm.raw_empty[r]);
