@@ -28,18 +28,21 @@
 // (N = 256 tokens), 128-byte-swizzled tiles loaded by TMA.  The accumulator is
 // D[weight row][token]; the epilogue writes Y[token][weight row].
 //
-// Roles (one persistent CTA per SM, 14 warps, tiles of 128 weight rows x 256
+// Roles (one persistent CTA per SM, 16 warps, tiles of 128 weight rows x 256
 // tokens):
-//   warp 0      TMA producer: activation K-blocks (two 128-byte boxes of 256
-//               rows), packed weight K-blocks and their raw scale tiles.
+//   warp 0      activation producer: TMA of 128-byte-wide boxes of the tile's
+//               256 token rows into a 4-stage ring released by MMA commits.
 //   warp 1      TMEM owner (512 columns: accumulator 256, plane ring 8 x 24),
 //               MMA issuer.
-//   warps 2-9   converters, one weight row per thread (TMEM lane), two warps
+//   warp 2      weight producer: packed weight K-blocks and their raw scale
+//               tiles into a 4-stage ring released by the converters, so the
+//               weights run ahead of the activations.
+//   warps 4-11  converters, one weight row per thread (TMEM lane), two warps
 //               per lane quarter taking the even and the odd K steps: per step,
 //               32 codes -> three planes of 32 E5M2 bytes -> tcgen05.st.  The
 //               plane tables of every scale byte are built once per CTA in
 //               shared memory.
-//   warps 10-13 epilogue: TMEM -> registers, x alpha, BF16 RNE, store.
+//   warps 12-15 epilogue: TMEM -> registers, x alpha, BF16 RNE, store.
 // Requires K % 256 == 0 (TMA of the scale tiles).
 #pragma once
 #include <cuda_bf16.h>
@@ -56,27 +59,32 @@ using via_fp8::warp_wait;
 
 constexpr int BW = 128;               // weight rows per tile (TMEM lanes, the MMA's M)
 constexpr int BT = 256;               // tokens per tile (the MMA's N)
-constexpr int BK = 256;               // codes per raw K-block
-constexpr int STEPS = BK / 32;        // K = 32 MMA steps per K-block
-constexpr int RSTAGES = 2;            // raw K-block ring
+constexpr int BK = 256;               // codes per weight K-block
+constexpr int STEPS = BK / 32;        // K = 32 MMA steps per weight K-block
+constexpr int ASTAGES = 4;            // activation ring, 128 bytes of K (4 steps) per stage
+constexpr int WSTAGES = 4;            // weight ring, one K-block per stage
 constexpr int PLANES = 3;             // signed digits of a scale, at most
 constexpr int NSLOT = 8;              // TMEM plane-slot ring, one K step each
 constexpr int SLOT_COLS = PLANES * 8; // 32 bytes of K per lane = 8 columns per plane
 constexpr int ACC_COLS = BT;          // FP32 accumulator columns
 constexpr int TMEM_COLS = 512;
 constexpr int CONV_WARPS = 8, EPI_WARPS = 4;  // two converter warps per TMEM lane quarter
-constexpr int NUM_THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
+constexpr int CONV_PER_Q = CONV_WARPS / 4;    // ... taking every CONV_PER_Q-th K step
+constexpr int FIRST_CONV = 4;                 // warps 0-3: producers, MMA, one spare
+constexpr int NUM_THREADS = 32 * (FIRST_CONV + CONV_WARPS + EPI_WARPS);
 static_assert(ACC_COLS + NSLOT * SLOT_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(NSLOT == STEPS, "one TMEM slot per K step of a block");
 
 enum Role { ROLE_PRODUCER = 1, ROLE_MMA = 2, ROLE_CONV = 3, ROLE_EPI = 4, ROLE_DRAIN = 5 };
 
 struct Smem {
-    alignas(1024) uint8_t act[RSTAGES][2][BT * 128];  // E4M3 activations, two swizzled boxes
-    alignas(1024) uint8_t w[RSTAGES][BW * 128];       // packed FP4 weights, swizzled
-    alignas(16) uint8_t sw[RSTAGES][BW * 16];         // weight scales [row][16 groups]
-    uint4 ptab[128][PLANES];                          // plane tables per scale byte (lo, hi, sgn)
-    uint64_t raw_full[RSTAGES], raw_empty[RSTAGES];
+    alignas(1024) uint8_t act[ASTAGES][BT * 128];     // E4M3 activations, 128-byte swizzled
+    alignas(1024) uint8_t w[WSTAGES][BW * 128];       // packed FP4 weights, swizzled
+    alignas(16) uint8_t sw[WSTAGES][BW * 16];         // weight scales [row][16 groups]
+    uint4 ptab01[128];                                // plane tables per scale byte: planes 0, 1
+    uint2 ptab2[128];                                 // ... and plane 2
+    uint64_t act_full[ASTAGES], act_empty[ASTAGES];
+    uint64_t w_full[WSTAGES], w_empty[WSTAGES];
     uint64_t slot_full[NSLOT], slot_empty[NSLOT];
     uint64_t acc_full, acc_empty;
     uint64_t drain;
@@ -84,7 +92,8 @@ struct Smem {
     int abort;
 };
 constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
-constexpr uint32_t RAW_BYTES = BT * 256 + BW * 128 + BW * 16;
+constexpr uint32_t ACT_BYTES = BT * 128;
+constexpr uint32_t W_BYTES = BW * 128 + BW * 16;
 
 // kind::f8f6f4 instruction descriptor: F32 accumulator, A and B formats
 // (0 = E4M3, 1 = E5M2), both K-major, M x N.
@@ -116,15 +125,18 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// One plane of one group: an 8-entry byte table T[c] = E5M2(e2m1(c) * 2^p) for
-// the magnitude codes c = 0..7 (T[0] = 0), as two words for byte_perm, and the
-// digit's sign as a byte mask.  With base = (p + 14) << 2 the E5M2 bytes are
-//   c=1 (0.5): base         c=2 (1): base + 4    c=3 (1.5): base + 6
-//   c=4 (2):   base + 8     c=5 (3): base + 10   c=6 (4):   base + 12
-//   c=7 (6):   base + 14
-// (exponent field p + 14 + e2m1 exponent, mantissa bit of the code in bit 1).
+// One plane of one group: an 8-entry byte table T[c] = E5M2(sigma * e2m1(c) *
+// 2^p) for the magnitude codes c = 0..7, as two words for byte_perm.  With
+// base = (p + 14) << 2 the E5M2 magnitudes are
+//   c=0: 0                  c=1 (0.5): base      c=2 (1): base + 4
+//   c=3 (1.5): base + 6     c=4 (2): base + 8    c=5 (3): base + 10
+//   c=6 (4): base + 12      c=7 (6): base + 14
+// (exponent field p + 14 + e2m1 exponent, mantissa bit of the code in bit 1),
+// and the digit's sign sigma sits in bit 7 of every entry (so T[0] may be -0).
+// A plane the scale does not use is all 0x80: -0 for every code.  The code's
+// own sign is XORed in afterwards.
 struct PlaneTable {
-    uint32_t lo, hi, sgn;
+    uint32_t lo, hi;
 };
 
 __device__ __forceinline__ void plane_tables(uint32_t sb, PlaneTable (&t)[PLANES]) {
@@ -140,13 +152,12 @@ __device__ __forceinline__ void plane_tables(uint32_t sb, PlaneTable (&t)[PLANES
             const int ti = __ffs(d) - 1;
             d &= d - 1;
             const uint32_t base = (uint32_t)(ti + b + 14) << 2;
-            t[i].lo = base * 0x01010100u + 0x06040000u;
-            t[i].hi = base * 0x01010101u + 0x0E0C0A08u;
-            t[i].sgn = ((neg >> ti) & 1u) ? 0x80808080u : 0u;
+            const uint32_t sgn = ((neg >> ti) & 1u) ? 0x80808080u : 0u;
+            t[i].lo = (base * 0x01010100u + 0x06040000u) | sgn;
+            t[i].hi = (base * 0x01010101u + 0x0E0C0A08u) | sgn;
         } else {
-            t[i].lo = 0u;
-            t[i].hi = 0u;
-            t[i].sgn = 0u;
+            t[i].lo = 0x80808080u;
+            t[i].hi = 0x80808080u;
         }
     }
 }
@@ -161,8 +172,18 @@ __device__ __forceinline__ void convert8_planes(uint32_t w, const PlaneTable (&t
     const uint32_t sg_hi = __byte_perm(0x8000u, 0u, (w >> 19) & 0x1111u);
 #pragma unroll
     for (int i = 0; i < PLANES; ++i) {
-        out[i][0] = __byte_perm(t[i].lo, t[i].hi, sel_lo) | (sg_lo ^ t[i].sgn);
-        out[i][1] = __byte_perm(t[i].lo, t[i].hi, sel_hi) | (sg_hi ^ t[i].sgn);
+        out[i][0] = __byte_perm(t[i].lo, t[i].hi, sel_lo) ^ sg_lo;
+        out[i][1] = __byte_perm(t[i].lo, t[i].hi, sel_hi) ^ sg_hi;
+    }
+}
+
+// A producer that has given up waits (bounded) for the copies it started.
+__device__ __forceinline__ void drain_copies(uint64_t* full, int stages, int it) {
+    for (int j = max(0, it - stages); j < it; ++j) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[j % stages], (j / stages) & 1) &&
+               globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
     }
 }
 
@@ -181,12 +202,16 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
     volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < RSTAGES; ++s) {
-            mbar_init(&sm.raw_full[s], 1);
-            mbar_init(&sm.raw_empty[s], CONV_WARPS + 1);  // converters + the MMA's commit
+        for (int s = 0; s < ASTAGES; ++s) {
+            mbar_init(&sm.act_full[s], 1);
+            mbar_init(&sm.act_empty[s], 1);           // the MMA's commit
+        }
+        for (int s = 0; s < WSTAGES; ++s) {
+            mbar_init(&sm.w_full[s], 1);
+            mbar_init(&sm.w_empty[s], CONV_WARPS);    // every converter warp
         }
         for (int s = 0; s < NSLOT; ++s) {
-            mbar_init(&sm.slot_full[s], CONV_WARPS / 2);  // the four warps of the step's parity
+            mbar_init(&sm.slot_full[s], 4);  // the step's converter warp of each lane quarter
             mbar_init(&sm.slot_empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
@@ -201,8 +226,8 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
     if (threadIdx.x < 128) {  // the plane tables of scale byte threadIdx.x
         PlaneTable t[PLANES];
         plane_tables(threadIdx.x, t);
-#pragma unroll
-        for (int i = 0; i < PLANES; ++i) sm.ptab[threadIdx.x][i] = make_uint4(t[i].lo, t[i].hi, t[i].sgn, 0u);
+        sm.ptab01[threadIdx.x] = make_uint4(t[0].lo, t[0].hi, t[1].lo, t[1].hi);
+        sm.ptab2[threadIdx.x] = make_uint2(t[2].lo, t[2].hi);
     }
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, TMEM_COLS);
@@ -214,60 +239,70 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
     const uint32_t tmem = sm.tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ activation producer
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+                int tt, tw;
+                tile_coords(tile, num_t, num_w, tt, tw);
+                for (int j = 0; j < 2 * num_kb; ++j, ++it) {
+                    const int a = it % ASTAGES;
+                    if (!mbar_wait(&sm.act_empty[a], ((it / ASTAGES) & 1) ^ 1, abort, ROLE_PRODUCER))
+                        goto act_done;
+                    mbar_arrive_expect_tx(&sm.act_full[a], ACT_BYTES);
+                    tma_load_2d(sm.act[a], &tmA, &sm.act_full[a], j * 128, tt * BT);
+                }
+            }
+        act_done:
+            if (*abort) drain_copies(sm.act_full, ASTAGES, it);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ weight producer
         if (lane == 0) {
             int it = 0;
             for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
                 int tt, tw;
                 tile_coords(tile, num_t, num_w, tt, tw);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int r = it % RSTAGES;
-                    if (!mbar_wait(&sm.raw_empty[r], ((it / RSTAGES) & 1) ^ 1, abort, ROLE_PRODUCER))
-                        goto producer_done;
-                    mbar_arrive_expect_tx(&sm.raw_full[r], RAW_BYTES);
-                    tma_load_2d(sm.act[r][0], &tmA, &sm.raw_full[r], kb * 256, tt * BT);
-                    tma_load_2d(sm.act[r][1], &tmA, &sm.raw_full[r], kb * 256 + 128, tt * BT);
-                    tma_load_2d(sm.w[r], &tmB, &sm.raw_full[r], kb * 128, tw * BW);
-                    tma_load_2d(sm.sw[r], &tmSB, &sm.raw_full[r], kb * 16, tw * BW);
+                    const int r = it % WSTAGES;
+                    if (!mbar_wait(&sm.w_empty[r], ((it / WSTAGES) & 1) ^ 1, abort, ROLE_PRODUCER))
+                        goto w_done;
+                    mbar_arrive_expect_tx(&sm.w_full[r], W_BYTES);
+                    tma_load_2d(sm.w[r], &tmB, &sm.w_full[r], kb * 128, tw * BW);
+                    tma_load_2d(sm.sw[r], &tmSB, &sm.w_full[r], kb * 16, tw * BW);
                 }
             }
-        producer_done:
-            if (*abort) {
-                for (int j = max(0, it - RSTAGES); j < it; ++j) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(&sm.raw_full[j % RSTAGES], (j / RSTAGES) & 1) &&
-                           globaltimer_ns() - t0 < kWaitLimitNs) {
-                    }
-                }
-            }
+        w_done:
+            if (*abort) drain_copies(sm.w_full, WSTAGES, it);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_f8f6f4(BW, BT, /*A E5M2*/ 1u, /*B E4M3*/ 0u);
-            int it = 0, st = 0, tc = 0;
+            int ait = 0, it = 0, tc = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
                 // the epilogue has read the previous tile's accumulator
                 if (!mbar_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
                 tc_fence_after();
                 for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
-                    const int r = it % RSTAGES;
-                    if (!mbar_wait(&sm.raw_full[r], (it / RSTAGES) & 1, abort, ROLE_MMA)) { ok = false; break; }
-                    for (int h = 0; h < STEPS; ++h, ++st) {
-                        const int s = st % NSLOT;
-                        if (!mbar_wait(&sm.slot_full[s], (st / NSLOT) & 1, abort, ROLE_MMA)) { ok = false; break; }
-                        tc_fence_after();
-                        // B: the K = 32 slice of the 256 activation rows (128-byte swizzle)
-                        const uint64_t bdesc =
-                            desc_kmajor_sw128(smem_u32(sm.act[r][h >> 2]) + (h & 3) * 32);
-                        const uint32_t a0 = tmem + ACC_COLS + s * SLOT_COLS;
+                    for (int half = 0; half < 2 && ok; ++half, ++ait) {
+                        const int a = ait % ASTAGES;
+                        if (!mbar_wait(&sm.act_full[a], (ait / ASTAGES) & 1, abort, ROLE_MMA)) { ok = false; break; }
+                        for (int hh = 0; hh < 4; ++hh) {
+                            const int h = 4 * half + hh;  // K step of the block = TMEM slot
+                            if (!mbar_wait(&sm.slot_full[h], it & 1, abort, ROLE_MMA)) { ok = false; break; }
+                            tc_fence_after();
+                            // B: the K = 32 slice of the 256 activation rows (128-byte swizzle)
+                            const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sm.act[a]) + hh * 32);
+                            const uint32_t a0 = tmem + ACC_COLS + h * SLOT_COLS;
 #pragma unroll
-                        for (int i = 0; i < PLANES; ++i)
-                            mma_f8f6f4_ts(tmem, a0 + i * 8, bdesc, idesc, (kb | h | i) != 0);
-                        mma_commit(&sm.slot_empty[s]);
+                            for (int i = 0; i < PLANES; ++i)
+                                mma_f8f6f4_ts(tmem, a0 + i * 8, bdesc, idesc, (kb | h | i) != 0);
+                            mma_commit(&sm.slot_empty[h]);
+                        }
+                        if (ok) mma_commit(&sm.act_empty[a]);  // this stage's activations are read
                     }
-                    if (ok) mma_commit(&sm.raw_empty[r]);  // the activations of this stage are read
                 }
                 if (ok) mma_commit(&sm.acc_full);
             }
@@ -280,35 +315,35 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
                 }
             }
         }
-    } else if (warp < 2 + CONV_WARPS) {
+    } else if (warp >= FIRST_CONV && warp < FIRST_CONV + CONV_WARPS) {
         // ------------------------------------------------------------ converters
-        const int q = warp & 3;                 // TMEM lane quarter this warp may access
-        const int par = (warp - 2) >> 2;        // this warp's K steps: h = par, par + 2, ...
-        const int row = 32 * q + lane;          // weight row within the tile
+        const int q = warp & 3;                      // TMEM lane quarter this warp may access
+        const int par = (warp - FIRST_CONV) >> 2;    // K steps h = par, par + CONV_PER_Q, ...
+        const int row = 32 * q + lane;               // weight row within the tile
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + ACC_COLS;
         int it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
-                const int r = it % RSTAGES;
-                if (!warp_wait(&sm.raw_full[r], (it / RSTAGES) & 1, abort, ROLE_CONV)) { ok = false; break; }
+                const int r = it % WSTAGES;
+                if (!warp_wait(&sm.w_full[r], (it / WSTAGES) & 1, abort, ROLE_CONV)) { ok = false; break; }
                 const uint4 sbq = *reinterpret_cast<const uint4*>(sm.sw[r] + row * 16);
                 const uint32_t sbw[4] = {sbq.x, sbq.y, sbq.z, sbq.w};
 #pragma unroll 1
-                for (int h = par; h < STEPS; h += 2) {
-                    // K step h of the block uses TMEM slot h (STEPS == NSLOT)
-                    // codes 32h .. 32h+31 of the row: 16 bytes, chunk h of the 128-byte
-                    // swizzled row; groups 2h and 2h+1
+                for (int h = par; h < STEPS; h += CONV_PER_Q) {
+                    // K step h of the block uses TMEM slot h (STEPS == NSLOT): codes
+                    // 32h .. 32h+31 of the row, 16 bytes, chunk h of the 128-byte swizzled
+                    // row; groups 2h and 2h+1
                     const uint4 qb = *reinterpret_cast<const uint4*>(
                         sm.w[r] + row * 128 + ((h ^ (row & 7)) << 4));
                     const uint32_t sb0 = (sbw[h >> 1] >> (16 * (h & 1))) & 0x7Fu;
                     const uint32_t sb1 = (sbw[h >> 1] >> (16 * (h & 1) + 8)) & 0x7Fu;
                     PlaneTable t0[PLANES], t1[PLANES];
-#pragma unroll
-                    for (int i = 0; i < PLANES; ++i) {
-                        const uint4 a = sm.ptab[sb0][i], b = sm.ptab[sb1][i];
-                        t0[i].lo = a.x; t0[i].hi = a.y; t0[i].sgn = a.z;
-                        t1[i].lo = b.x; t1[i].hi = b.y; t1[i].sgn = b.z;
+                    {
+                        const uint4 a01 = sm.ptab01[sb0], b01 = sm.ptab01[sb1];
+                        const uint2 a2 = sm.ptab2[sb0], b2 = sm.ptab2[sb1];
+                        t0[0] = {a01.x, a01.y}; t0[1] = {a01.z, a01.w}; t0[2] = {a2.x, a2.y};
+                        t1[0] = {b01.x, b01.y}; t1[1] = {b01.z, b01.w}; t1[2] = {b2.x, b2.y};
                     }
                     uint32_t o0[PLANES][2], o1[PLANES][2], o2[PLANES][2], o3[PLANES][2];
                     convert8_planes(qb.x, t0, o0);
@@ -329,10 +364,10 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
                     if (lane == 0) mbar_arrive(&sm.slot_full[h]);
                 }
                 __syncwarp();
-                if (ok && lane == 0) mbar_arrive(&sm.raw_empty[r]);
+                if (ok && lane == 0) mbar_arrive(&sm.w_empty[r]);  // this K-block's weights are read
             }
         }
-    } else {
+    } else if (warp >= FIRST_CONV + CONV_WARPS) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
