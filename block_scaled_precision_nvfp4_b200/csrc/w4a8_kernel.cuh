@@ -166,10 +166,12 @@ __device__ __forceinline__ void plane_tables(uint32_t sb, PlaneTable (&t)[PLANES
 // bytes in k order (byte j of the first word = code j).
 __device__ __forceinline__ void convert8_planes(uint32_t w, const PlaneTable (&t)[PLANES],
                                                 uint32_t (&out)[PLANES][2]) {
-    const uint32_t sel_lo = w & 0x7777u, sel_hi = (w >> 16) & 0x7777u;
+    // byte_perm reads the low 16 bits of its selector: four nibbles
+    const uint32_t sel_lo = w & 0x77777777u, sel_hi = sel_lo >> 16;
     // 0x80 in byte j where code j is negative: byte_perm of (byte 0 = 0, byte 1 = 0x80)
-    const uint32_t sg_lo = __byte_perm(0x8000u, 0u, (w >> 3) & 0x1111u);
-    const uint32_t sg_hi = __byte_perm(0x8000u, 0u, (w >> 19) & 0x1111u);
+    const uint32_t sgn = (w >> 3) & 0x11111111u;
+    const uint32_t sg_lo = __byte_perm(0x8000u, 0u, sgn);
+    const uint32_t sg_hi = __byte_perm(0x8000u, 0u, sgn >> 16);
 #pragma unroll
     for (int i = 0; i < PLANES; ++i) {
         out[i][0] = __byte_perm(t[i].lo, t[i].hi, sel_lo) ^ sg_lo;
@@ -279,6 +281,9 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_f8f6f4(BW, BT, /*A E5M2*/ 1u, /*B E4M3*/ 0u);
+            // descriptor of stage 0's first K slice; stage a and slice hh add their offsets
+            // (in 16-byte units) to the start-address field
+            const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(sm.act[0]));
             int ait = 0, it = 0, tc = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
@@ -294,7 +299,7 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
                             if (!mbar_wait(&sm.slot_full[h], it & 1, abort, ROLE_MMA)) { ok = false; break; }
                             tc_fence_after();
                             // B: the K = 32 slice of the 256 activation rows (128-byte swizzle)
-                            const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sm.act[a]) + hh * 32);
+                            const uint64_t bdesc = bdesc0 + (uint64_t)(a * (BT * 128 / 16) + hh * 2);
                             const uint32_t a0 = tmem + ACC_COLS + h * SLOT_COLS;
 #pragma unroll
                             for (int i = 0; i < PLANES; ++i)
