@@ -29,7 +29,7 @@ __all__ = [
     "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
     "gemm_nvfp4_w4a4_packed", "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
     "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "nvfp4_fp4_fallback",
-    "nvfp4_node_exec", "C_FUNCTIONS",
+    "nvfp4_node_exec", "moe_route", "moe_permute_rows", "moe_combine", "C_FUNCTIONS",
 ]
 
 
@@ -97,6 +97,10 @@ C_FUNCTIONS = {
     "nvfp4_pack_scales_grouped": (_I, [_P, _P, _I, _I, _P, _P]),
     "gemm_nvfp4_w4a4_grouped_packed": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
     "nvfp4_quantize_workspace_bytes": (_Z, []),
+    "nvfp4_moe_route_workspace_bytes": (_Z, [_I, _I]),
+    "nvfp4_moe_route": (_I, [_P, _I, _I, _P, _P, _P, _P, _Z, _P]),
+    "nvfp4_moe_permute_rows": (_I, [_P, _Z, _I, _I, _I, _P, _P, _P]),
+    "nvfp4_moe_combine": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _P]),
     "nvfp4_quantize_bf16": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "nvfp4_quantize_bf16_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _P]),
 }
@@ -449,4 +453,63 @@ def gemm_nvfp4_w4a4_grouped_packed(A, sA_packed, gA, W, sW_packed, gW, offsets, 
         pa, sA_packed.data_ptr(), float(gA), pw, sW_packed.data_ptr(),
         ctypes.cast(gws, ctypes.c_void_p), ctypes.cast(off, ctypes.c_void_p), E, py, N, K,
         _stream_ptr(stream)))
+    return out
+
+
+# --- MoE dispatch and combine around the grouped product ---------------------------
+
+def moe_route(expert_ids, E, workspace=None, stream=None):
+    """Top-k routing -> (offsets [E+1], dest [P], src [P]), device int32.
+
+    expert_ids: CUDA int32 [T, k] (or [P]); pair p = t*k + j.  Rows of expert e in
+    the grouped order are offsets[e] .. offsets[e+1]-1, pairs in their order p."""
+    torch = _torch()
+    ids = expert_ids.reshape(-1)
+    P = ids.numel()
+    pid = _dev_tensor(ids, torch.int32, (P,), "expert_ids")
+    lib = load_library()
+    need = int(lib.nvfp4_moe_route_workspace_bytes(P, int(E)))
+    if need == 0:
+        raise ValueError(f"E must be in [1, 256] (got {E})")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=ids.device)
+    offsets = torch.empty(int(E) + 1, dtype=torch.int32, device=ids.device)
+    dest = torch.empty(max(P, 1), dtype=torch.int32, device=ids.device)
+    src = torch.empty(max(P, 1), dtype=torch.int32, device=ids.device)
+    _err(lib.nvfp4_moe_route(pid, P, int(E), offsets.data_ptr(), dest.data_ptr(), src.data_ptr(),
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             _stream_ptr(stream)))
+    return offsets, dest[:P], src[:P]
+
+
+def moe_permute_rows(x, src, k, out=None, stream=None):
+    """Rows of x (CUDA uint8 [rows, row_bytes], token order) -> expert-grouped order:
+    out[r] = x[src[r] // k], one row per pair."""
+    torch = _torch()
+    rows, row_bytes = x.shape
+    P = src.numel()
+    px = _dev_tensor(x, torch.uint8, (rows, row_bytes), "x")
+    ps = _dev_tensor(src, torch.int32, (P,), "src")
+    if out is None:
+        out = torch.empty((P, row_bytes), dtype=torch.uint8, device=x.device)
+    po = _dev_tensor(out, torch.uint8, (P, row_bytes), "out")
+    _err(load_library().nvfp4_moe_permute_rows(px, row_bytes, rows, P, int(k), ps, po,
+                                               _stream_ptr(stream)))
+    return out
+
+
+def moe_combine(Yg, dest, weights, T, k, out=None, stream=None):
+    """Y[t] = BF16(sum_j weights[t, j] * Yg[dest[t*k + j]]), FP32 in j order.
+    Yg: CUDA bf16 [P, N] in the expert-grouped order; weights: float32 [T, k] or None."""
+    torch = _torch()
+    P, N = Yg.shape
+    py = _dev_tensor(Yg, torch.bfloat16, (P, N), "Yg")
+    pd = _dev_tensor(dest.reshape(-1), torch.int32, (T * k,), "dest")
+    pw = None
+    if weights is not None:
+        pw = _dev_tensor(weights.reshape(-1), torch.float32, (T * k,), "weights")
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=Yg.device)
+    po = _dev_tensor(out, torch.bfloat16, (T, N), "out")
+    _err(load_library().nvfp4_moe_combine(py, P, pd, pw, int(T), int(k), N, po, _stream_ptr(stream)))
     return out

@@ -25,6 +25,7 @@
 #include "grouped_kernel.cuh"
 #include "grouped_pair_kernel.cuh"
 #include "quantize_kernel.cuh"
+#include "moe_kernel.cuh"
 
 namespace {
 
@@ -357,7 +358,9 @@ nvfp4_status nvfp4_check_device_error(void* stream) {
     if (v == 0) return ok();
     e = cudaMemcpyToSymbol(nvfp4::g_device_error, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
-    return fail(NVFP4_ERR_DEVICE_TIMEOUT, "a kernel wait expired (role %d)", (v >> 8) & 0xFF);
+    if (v & 0xFF)
+        return fail(NVFP4_ERR_DEVICE_TIMEOUT, "a kernel wait expired (role %d)", (v >> 8) & 0xFF);
+    return fail(NVFP4_ERR_INVALID_ARG, "a routed expert id was outside [0, E)");
 }
 
 // ------------------------------------------------------------------------- W4A4
@@ -664,6 +667,93 @@ nvfp4_status gemm_nvfp4_w4a8(const uint8_t* A_fp8, float gA, const uint8_t* W, c
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launching w4a8_kernel");
     return ok();
+}
+
+// ------------------------------------------------------------------------- MoE
+namespace {
+int route_chunks(int P) {
+    const int c = (P + nvfp4::moe::ROUTE_THREADS - 1) / nvfp4::moe::ROUTE_THREADS;
+    return c < nvfp4::moe::MAX_CHUNKS ? c : nvfp4::moe::MAX_CHUNKS;
+}
+}  // namespace
+
+size_t nvfp4_moe_route_workspace_bytes(int num_pairs, int E) {
+    if (num_pairs < 0 || E < 1 || E > nvfp4::moe::MAX_EXPERTS) return 0;
+    return (size_t)2 * route_chunks(num_pairs) * E * sizeof(int32_t) + 16;
+}
+
+nvfp4_status nvfp4_moe_route(const int32_t* expert_ids, int num_pairs, int E, int32_t* offsets,
+                             int32_t* dest, int32_t* src, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    namespace mo = nvfp4::moe;
+    if (num_pairs < 0) return fail(NVFP4_ERR_INVALID_ARG, "num_pairs must be >= 0 (got %d)", num_pairs);
+    if (E < 1 || E > mo::MAX_EXPERTS)
+        return fail(NVFP4_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", mo::MAX_EXPERTS, E);
+    if (!offsets || (num_pairs > 0 && (!expert_ids || !dest || !src || !workspace)))
+        return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(workspace) && num_pairs > 0)
+        return fail(NVFP4_ERR_MISALIGNED, "the workspace must be 16-byte aligned");
+    const size_t need = nvfp4_moe_route_workspace_bytes(num_pairs, E);
+    if (num_pairs > 0 && workspace_bytes < need)
+        return fail(NVFP4_ERR_INVALID_ARG, "route workspace of %zu bytes is too small (need %zu)",
+                    workspace_bytes, need);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (num_pairs == 0) {
+        e = cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "clearing the expert offsets");
+    }
+    // pairs with an out-of-range id are placed nowhere: their dest stays -1, and rows
+    // no pair lands on keep src = -1
+    if ((e = cudaMemsetAsync(dest, 0xFF, (size_t)num_pairs * sizeof(int32_t), s)) != cudaSuccess ||
+        (e = cudaMemsetAsync(src, 0xFF, (size_t)num_pairs * sizeof(int32_t), s)) != cudaSuccess)
+        return cuda_fail(e, "clearing the route maps");
+    const int C = route_chunks(num_pairs);
+    const int chunk = (num_pairs + C - 1) / C;
+    int32_t* counts = static_cast<int32_t*>(workspace);
+    int32_t* base = counts + (size_t)C * E;
+    mo::route_count_kernel<<<C, mo::ROUTE_THREADS, 0, s>>>(expert_ids, num_pairs, E, chunk, counts);
+    mo::route_scan_kernel<<<1, mo::MAX_EXPERTS, 0, s>>>(counts, C, E, base, offsets);
+    mo::route_rank_kernel<<<C, mo::ROUTE_THREADS, 0, s>>>(expert_ids, num_pairs, E, chunk, base, dest,
+                                                          src);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "launching the route kernels");
+}
+
+nvfp4_status nvfp4_moe_permute_rows(const void* in, size_t row_bytes, int in_rows, int num_pairs,
+                                    int k, const int32_t* src, void* out, void* stream) {
+    if (in_rows < 0 || num_pairs < 0 || k < 1)
+        return fail(NVFP4_ERR_INVALID_ARG, "in_rows, num_pairs >= 0 and k >= 1 required");
+    if (row_bytes == 0 || row_bytes % 16 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16 (got %zu)",
+                    row_bytes);
+    if (num_pairs == 0) return ok();
+    if (!in || !src || !out) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(in) || !aligned16(out))
+        return fail(NVFP4_ERR_MISALIGNED, "in and out must be 16-byte aligned");
+    nvfp4::moe::permute_rows_kernel<<<(num_pairs + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(in), row_bytes, in_rows, num_pairs, k, src,
+        static_cast<uint8_t*>(out));
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "launching permute_rows_kernel");
+}
+
+nvfp4_status nvfp4_moe_combine(const void* Yg, int num_pairs, const int32_t* dest,
+                               const float* weights, int T, int k, int N, void* Y, void* stream) {
+    if (T < 0 || num_pairs < 0 || k < 1 || N < 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "T, num_pairs, N >= 0 and k >= 1 required");
+    if (N % 8 != 0) return fail(NVFP4_ERR_INVALID_ARG, "N must be a multiple of 8 (got %d)", N);
+    if (T == 0 || N == 0) return ok();
+    if (!dest || !Y || (num_pairs > 0 && !Yg)) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(Y) || (Yg && !aligned16(Yg)))
+        return fail(NVFP4_ERR_MISALIGNED, "Yg and Y must be 16-byte aligned");
+    const int cols = (N / 8 + 255) / 256;
+    const dim3 grid(cols, T < 65535 ? T : 65535);
+    nvfp4::moe::combine_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(Yg), num_pairs, dest, weights, T, k, N,
+        static_cast<__nv_bfloat16*>(Y));
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "launching combine_kernel");
 }
 
 // ------------------------------------------------------------------------- W4A16

@@ -271,6 +271,50 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a8(const uint8_t* A_fp8, float gA, const uin
                                        const uint8_t* sW, float gW, void* Y_bf16, int M, int N,
                                        int K, void* stream);
 
+/* ---- MoE dispatch and combine around the grouped product ------------------
+ * (page 2, the MegaMoE swap-AB kernel: tokens are dispatched to their experts,
+ * run through one grouped GEMM, and combined back with their routing weights.)
+ * A "pair" is one (token t, slot j) of a top-k routing, numbered p = t*k + j. */
+
+/* Workspace bytes of nvfp4_moe_route for num_pairs pairs and E experts (0 for
+ * num_pairs < 0 or E outside [1, 256]). */
+NVFP4_API size_t nvfp4_moe_route_workspace_bytes(int num_pairs, int E);
+
+/* Route: expert_ids [num_pairs] (device int32, pair p's expert) ->
+ *   offsets [E+1]       rows of expert e are offsets[e] .. offsets[e+1]-1 of the
+ *                       expert-grouped order (the `offsets` of the grouped GEMM);
+ *   dest [num_pairs]    pair p's row in that order;
+ *   src  [num_pairs]    the pair on grouped row r (src[dest[p]] = p).
+ * Inside an expert, pairs keep their order p (stable, hence deterministic).
+ * All arrays are device memory owned by the caller; workspace is device memory
+ * of nvfp4_moe_route_workspace_bytes bytes, 16-byte aligned, overwritten.  An id
+ * outside [0, E) is placed nowhere (its dest stays -1, and offsets[E] counts only
+ * placed pairs) and makes the next nvfp4_check_device_error return
+ * NVFP4_ERR_INVALID_ARG.  E in [1, 256]; num_pairs == 0 writes zero offsets. */
+NVFP4_API nvfp4_status nvfp4_moe_route(const int32_t* expert_ids, int num_pairs, int E,
+                                       int32_t* offsets, int32_t* dest, int32_t* src,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Permute (dispatch on one GPU): out[r] = in[src[r] / k] for r < num_pairs, whole
+ * rows of row_bytes bytes (a positive multiple of 16): the rows of a token's
+ * codes (K/2 bytes) or plain scales (K/16 bytes), in token order in `in`
+ * [in_rows][row_bytes], land in the expert-grouped order in `out`
+ * [num_pairs][row_bytes], one copy per pair.  A row whose src is outside
+ * [0, in_rows*k) is left untouched.  Device pointers, 16-byte aligned. */
+NVFP4_API nvfp4_status nvfp4_moe_permute_rows(const void* in, size_t row_bytes, int in_rows,
+                                              int num_pairs, int k, const int32_t* src,
+                                              void* out, void* stream);
+
+/* Combine: Y[t][n] = BF16( sum_{j<k} w[t][j] * Yg[dest[t*k+j]][n] ), the FP32
+ * products added in the order j = 0..k-1 and rounded once to nearest even.
+ * Yg is the grouped product's output, BF16 [num_pairs][N] in the expert-grouped
+ * order; weights is device FP32 [T][k] or NULL for all ones; Y is BF16 [T][N].
+ * A dest outside [0, num_pairs) contributes nothing.  N % 8 == 0; device
+ * pointers, Yg and Y 16-byte aligned. */
+NVFP4_API nvfp4_status nvfp4_moe_combine(const void* Yg_bf16, int num_pairs, const int32_t* dest,
+                                         const float* weights, int T, int k, int N, void* Y_bf16,
+                                         void* stream);
+
 /* W4A16: BF16 activations A_bf16 [M][K] (row-major) times NVFP4 weights, the
  * weights widened to BF16 in registers (exactly: an E2M1 value times an E4M3
  * scale has at most 6 significant bits), FP32 accumulation, gW applied in the
@@ -333,7 +377,9 @@ NVFP4_API const char* nvfp4_last_error(void);
 
 /* Synchronizes `stream`, then reads and clears the device error word that a
  * kernel sets when one of its bounded waits expires.  NVFP4_OK if clear,
- * NVFP4_ERR_DEVICE_TIMEOUT if set, NVFP4_ERR_CUDA if synchronization failed. */
+ * NVFP4_ERR_DEVICE_TIMEOUT if a wait expired, NVFP4_ERR_INVALID_ARG if the only
+ * record is an out-of-range expert id seen by nvfp4_moe_route, NVFP4_ERR_CUDA if
+ * synchronization failed. */
 NVFP4_API nvfp4_status nvfp4_check_device_error(void* stream);
 
 /* Library version string (static storage). */
