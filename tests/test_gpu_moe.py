@@ -133,3 +133,32 @@ def test_whole_moe_layer_against_the_oracle():
     rel = np.linalg.norm(bf16_to_f64(Y) - ref) / np.linalg.norm(ref)
     assert rel <= 2e-3 * np.sqrt(2), f"moe layer: relative Frobenius error {rel:.3e}"
     assert np.max(np.abs(bf16_to_f64(Y) - ref)) <= 1e-2 * np.max(np.abs(ref))
+
+
+def test_expert_parallel_path_on_one_rank_equals_the_direct_layer():
+    """ep.dispatch / ep.combine with the CUDA kernels and no process group (one rank
+    owning every expert) give the direct layer's output bit for bit."""
+    from block_scaled_precision_nvfp4_b200 import ep
+    rng = np.random.default_rng(11)
+    T, k, E, N, K = 300, 2, 4, 256, 512
+    ids = _ids(rng, T, k, E)
+    w = torch.from_numpy(rng.random((T, k)).astype(np.float32)).cuda()
+    A = wl.quantize_nvfp4(rng.standard_normal((T, K), dtype=np.float32))
+    experts = [wl.quantize_nvfp4(rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02))
+               for _ in range(E)]
+    Wc = torch.from_numpy(np.stack([e.codes for e in experts])).cuda()
+    Ws = torch.from_numpy(np.stack([e.scales for e in experts])).cuda()
+    gws = [e.g for e in experts]
+
+    def grouped(codes, scales, offsets):
+        return nv.gemm_nvfp4_w4a4_grouped(codes, scales, A.g, Wc, Ws, gws, offsets)
+
+    codes, scales = torch.from_numpy(A.codes).cuda(), torch.from_numpy(A.scales).cuda()
+    idd = torch.from_numpy(ids).cuda()
+    st = ep.dispatch(codes, scales, idd, E)
+    Y1 = ep.combine(grouped(st.codes, st.scales, st.local_offsets), st, w)
+    off, dest, src = nv.moe_route(idd, E)
+    gc, gs = nv.moe_permute_rows(codes, src, k), nv.moe_permute_rows(scales, src, k)
+    Y2 = nv.moe_combine(grouped(gc, gs, off.cpu().tolist()), dest, w, T, k)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
