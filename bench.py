@@ -479,28 +479,61 @@ def run_ours(args):
     if path == "quantize":  # no flops: whole-job GB/s of the algorithmic bytes
         value = world * alg_bytes / (t_ms * 1e-3) / 1e9
 
-    # end to end through the public API: pinned host inputs -> device -> call -> host result
+    # End to end through the public API, as a serving loop runs it: the weights are
+    # resident (loaded once, like model weights); every step copies its activations in
+    # from pinned host memory, runs, and copies its output back.  Two buffer sets and two
+    # copy streams let step i+1's input copy and step i-1's output copy overlap step i.
     e2e = None
     if not args.no_e2e:
-        hp = [torch.from_numpy(np.ascontiguousarray(h)).pin_memory() for h in host]
-        hY = torch.empty(tuple(Y.shape), dtype=Y.dtype).pin_memory()
-        e_steps = max(1, min(args.steps, 20))
+        n_act = {"quantize": 1, "w4a16": 1, "w4a8": 1}.get(path, 2)   # activations lead `host`
+        hp = [torch.from_numpy(np.ascontiguousarray(h)).pin_memory() for h in host[:n_act]]
+        dsets = [list(dv[:n_act]), [torch.empty_like(d) for d in dv[:n_act]]]
+        Ysets = [Y, torch.empty_like(Y)]
+        hYs = [torch.empty(tuple(Y.shape), dtype=Y.dtype).pin_memory() for _ in range(2)]
+        qsets = None
+        if path == "quantize":
+            qsets = [q_out, (Ysets[1], None, torch.empty_like(q_out[2]), torch.empty_like(q_out[3]))]
+        copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        comp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
+        e_steps = max(2, min(args.steps, 20))
 
-        def e2e_step():
-            for d, h in zip(dv, hp):
-                d.copy_(h, non_blocking=True)
+        def e2e_step(i):
+            nonlocal Y, xq, q_out, a16
+            b = i % 2
+            copy_in.wait_event(comp_done[b])          # step i-2 has finished reading set b
+            with torch.cuda.stream(copy_in):
+                for d, h in zip(dsets[b], hp):
+                    d.copy_(h, non_blocking=True)
+                in_ready[b].record(copy_in)
+            stream.wait_event(in_ready[b])
+            stream.wait_event(out_done[b])            # step i-2's output has left set b
+            dv[:n_act] = dsets[b]
+            Y = Ysets[b]
+            if path == "quantize":
+                xq, q_out = dsets[b][0].view(torch.bfloat16), qsets[b]
+            if path == "w4a16":
+                a16 = dsets[b][0].view(torch.bfloat16)
             step()
-            hY.copy_(Y, non_blocking=True)
+            comp_done[b].record(stream)
+            copy_out.wait_event(comp_done[b])
+            with torch.cuda.stream(copy_out):
+                hYs[b].copy_(Ysets[b], non_blocking=True)
+                out_done[b].record(copy_out)
 
-        for _ in range(2):
-            e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(e_steps):
-            e2e_step()
+        copy_in.wait_event(e0)
+        for i in range(e_steps):
+            e2e_step(i)
+        for b in range(2):
+            stream.wait_event(out_done[b])            # the last outputs are on the host
         e1.record(stream)
         torch.cuda.synchronize(dev)
         te = e0.elapsed_time(e1) / e_steps
@@ -508,12 +541,16 @@ def run_ours(args):
             tt = torch.tensor([te], dtype=torch.float64, device=dev)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             te = float(tt.item())
+        dv[:n_act] = dsets[0]
+        Y = Ysets[0]
         h2d = sum(x.numel() * x.element_size() for x in hp)
         e2e = {"value": (world * alg_bytes / (te * 1e-3) / 1e9 if path == "quantize"
                          else world * flops / (te * 1e-3) / 1e12),
                "unit": "GB/s" if path == "quantize" else "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hY.numel() * hY.element_size(),
-               "ms_per_step": te}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hYs[0].numel() * hYs[0].element_size(),
+               "ms_per_step": te,
+               "note": "weights resident; activations in and output out every step, "
+                       "two buffer sets, copies on two streams overlapping compute"}
 
     bf16_peak, hbm_peak, peak_src = peaks()
     kern_s = t_ms * 1e-3
