@@ -78,6 +78,9 @@ WORKLOADS = {
     "tiny": dict(path="w4a4", bound="tensor", desc="tiny W4A4 128x256x256"),
     "quantize": dict(path="quantize", bound="hbm",
                      desc="NVFP4 quantiser of the FFN-down activations, BF16 4096x14336"),
+    "moe": dict(path="moe", bound="tensor",
+                desc="MoE layer from BF16 tokens (quantise, route, permute, grouped W4A4, "
+                     "combine), 8 experts [14336,4096], 8192 tokens"),
 }
 
 
@@ -91,6 +94,8 @@ def make_workload(name):
         return wl.grouped_w4a4()
     if name == "quantize":
         return wl.activations_bf16()
+    if name == "moe":
+        return wl.moe_layer()
     if name == "w4a8":
         return wl.w4a8_ffn_down()
     return wl.ffn_down_w4a4()
@@ -110,6 +115,9 @@ def algorithmic(wl_, path):
         return flops, N * K // 2 + N * K // 16 + M * K + ybytes
     if path == "grouped":
         return flops, wl_.E * (N * K // 2 + N * K // 16) + M * (K // 2 + K // 16) + ybytes
+    if path == "moe":
+        # BF16 tokens in, every expert's weights once, Y out
+        return flops, M * K * 2 + wl_.E * (N * K // 2 + N * K // 16) + ybytes
     return flops, (M + N) * (K // 2 + K // 16) + ybytes
 
 
@@ -184,6 +192,20 @@ def _oracle_rows(wl_, rows):
     if wl_.N == 0:
         from oracle import quantize as oq
         oq.quantize_nvfp4_bf16(wl_.A_bf16[:rows])
+        return
+    if wl_.expert_ids is not None:
+        # the MoE layer on the first `rows` tokens: the quantiser (with the whole tensor's
+        # amax), each token through its expert, weight 1 (top-1)
+        from oracle import quantize as oq
+        amax = float(np.max(np.abs(oq.bf16_to_f32(wl_.A_bf16))))
+        codes, scales, g = oq.quantize_nvfp4_bf16(wl_.A_bf16[:rows], amax=amax)
+        ids = wl_.expert_ids[:rows, 0]
+        for e in range(wl_.E):
+            sel = np.nonzero(ids == e)[0]
+            if sel.size:
+                W = wl_.W_e[e]
+                oracle.gemm_w4a4(codes[sel], scales[sel], float(g), W.codes, W.scales, W.g,
+                                 sel.size, wl_.N, wl_.K)
         return
     if wl_.A_fp8 is not None:
         oracle.gemm_w4a8(wl_.A_fp8[:rows], wl_.gA, wl_.W.codes, wl_.W.scales, wl_.W.g, rows,
@@ -273,6 +295,8 @@ KERNEL_SOURCES = {
     "w4a8": ["w4a8_kernel.cuh", "via_fp8_kernel.cuh", "ptx.cuh"],
     "w4a16": ["w4a16_kernel.cuh"],
     "grouped": ["grouped_pair_kernel.cuh", "w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
+    "moe": ["grouped_pair_kernel.cuh", "w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh",
+            "moe_kernel.cuh", "quantize_kernel.cuh"],
     "quantize": ["quantize_kernel.cuh"],
 }
 
@@ -337,6 +361,8 @@ def run_ours(args):
         host = [wl_.A_bf16.view(np.int16), wl_.W.codes, wl_.W.scales]
     elif path == "w4a8":
         host = [wl_.A_fp8, wl_.W.codes, wl_.W.scales]
+    elif path == "moe":
+        host = [wl_.A_bf16.view(np.int16), wl_.expert_ids]     # per-step inputs only
     elif path == "grouped":
         Wc, Ws, gW = wlm.stack_experts(wl_)
         host = [wl_.A.codes, wl_.A.scales, Wc, Ws]
@@ -384,6 +410,51 @@ def run_ours(args):
         def plain_step():
             nv.gemm_nvfp4_w4a4_grouped(dv[0], dv[1], wl_.A.g, dv[2], dv[3], gw_list, offs,
                                        out=Y, stream=stream)
+    elif path == "moe":
+        # expert weights resident, their scales packed once (model load)
+        Wc_h, Ws_h, gW_h = wlm.stack_experts(wl_)
+        E = wl_.E
+        Wc_d, Ws_d = dev_(Wc_h), dev_(Ws_h)
+        gws = [float(x) for x in gW_h]
+        sw_packed = nv.nvfp4_pack_scales_grouped(Ws_d.view(E * N, K // 16),
+                                                 [e * N for e in range(E + 1)], K, stream=stream)
+        q_ws = torch.empty(16, dtype=torch.uint8, device=dev)
+        codes_b = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        scales_b = torch.empty((M, K // 16), dtype=torch.uint8, device=dev)
+        g_b = torch.empty(4, dtype=torch.float32, device=dev)
+        route_ws = torch.empty(nv.load_library().nvfp4_moe_route_workspace_bytes(M, E),
+                               dtype=torch.uint8, device=dev)
+        gc_b = torch.empty_like(codes_b)
+        gs_b = torch.empty_like(scales_b)
+        sa_b = torch.empty(nv.nvfp4_grouped_scale_layout_bytes([0] * E + [M], K) + 128 * (K // 16) * E,
+                           dtype=torch.uint8, device=dev)
+        Yg_b = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ones = torch.ones((M, 1), dtype=torch.float32, device=dev)
+
+        def step(stages=None):
+            def mark(i):
+                if stages is not None:
+                    stages[i].record(stream)
+            mark(0)
+            nv.nvfp4_quantize_bf16(dv[0].view(torch.bfloat16), plain=True, packed=False,
+                                   workspace=q_ws, stream=stream, out=(codes_b, scales_b, None, g_b))
+            mark(1)
+            off, dest, src = nv.moe_route(dv[1], E, workspace=route_ws, stream=stream)
+            mark(2)
+            nv.moe_permute_rows(codes_b, src, 1, out=gc_b, stream=stream)
+            nv.moe_permute_rows(scales_b, src, 1, out=gs_b, stream=stream)
+            mark(3)
+            # the grouped product plans its tiles on the host: offsets and gA come back
+            host_vals = torch.cat([off.to(torch.float64), g_b[:1].to(torch.float64)]).cpu()
+            offsets = [int(x) for x in host_vals[:E + 1]]
+            gA = float(host_vals[E + 1])
+            nv.nvfp4_pack_scales_grouped(gs_b, offsets, K, out=sa_b, stream=stream)
+            mark(4)
+            nv.gemm_nvfp4_w4a4_grouped_packed(gc_b, sa_b, gA, Wc_d, sw_packed, gws, offsets,
+                                              out=Yg_b, stream=stream)
+            mark(5)
+            nv.moe_combine(Yg_b, dest, ones, M, 1, out=Y, stream=stream)
+            mark(6)
     elif path == "w4a8":
         def step():
             nv.gemm_nvfp4_w4a8(dv[0], wl_.gA, dv[1], dv[2], wl_.W.g, out=Y, stream=stream)
@@ -407,7 +478,8 @@ def run_ours(args):
 
         def plain_step():
             nv.gemm_nvfp4_w4a4(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
-    launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2, "grouped": 2, "quantize": 2}.get(path, 1)
+    launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2, "grouped": 2, "quantize": 2,
+                         "moe": 10}.get(path, 1)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -444,6 +516,8 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     mids = ([torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
             if path in ("w4a4", "grouped") else None)
+    stage_ev = ([[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+                if path == "moe" else None)
     gstarts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     gends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with ClockSampler(dev.index) as clk:
@@ -452,6 +526,8 @@ def run_ours(args):
             starts[i].record(stream)
             if mids is not None:
                 step(mids[i])
+            elif stage_ev is not None:
+                step(stage_ev[i])
             else:
                 step()
             ends[i].record(stream)
@@ -573,7 +649,16 @@ def run_ours(args):
                  "gemm_packed_ms": statistics.median(gemm_ms),
                  "plain_scale_entry_ms": statistics.median(plain),
                  "plain_scale_entry_tflops": flops / (statistics.median(plain) * 1e-3) / 1e12}
+    if stage_ev is not None:
+        names = ["quantize", "route", "permute", "offsets_to_host_and_pack", "grouped_gemm", "combine"]
+        med = {n: statistics.median(ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev) * 1e3
+               for j, n in enumerate(names)}
+        kern_s = med["grouped_gemm"] * 1e-6
+        extra = {"stage_us": med,
+                 "permute_gbs": 2 * M * (K // 2 + K // 16) / (med["permute"] * 1e-6) / 1e9,
+                 "combine_gbs": 2 * M * N * 2 / (med["combine"] * 1e-6) / 1e9}
     kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel", "w4a8": "w4a8_kernel",
+                   "moe": "grouped_pair_kernel",
                    "w4a16": "w4a16_kernel", "grouped": "grouped_pair_kernel",
                    "quantize": "quantize_bf16_kernel (+ amax_bf16_kernel)"}[path]
     if spec["bound"] == "tensor_fp8":
@@ -646,6 +731,8 @@ def run_ours(args):
                   if path == "w4a16" else
                   "e4m3 x nvfp4(e2m1, e4m3 group scales) -> f32 accumulate -> bf16"
                   if path == "w4a8" else
+                  "bf16 -> nvfp4 -> grouped nvfp4 x nvfp4 -> f32 -> bf16 -> f32 combine -> bf16"
+                  if path == "moe" else
                   "nvfp4(e2m1 x e2m1, e4m3 group scales) -> f32 accumulate -> bf16"),
         "data": "synthetic",
         "config": {"workload": wl_.name, "M": M, "N": N, "K": K, "global_batch": world * M,

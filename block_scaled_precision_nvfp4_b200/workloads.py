@@ -47,6 +47,7 @@ class Workload:
     W: Operand | None = None          # NVFP4 weights [N, K]
     A_bf16: np.ndarray | None = None  # uint16 BF16 bit patterns [M, K] (W4A16)
     A_fp8: np.ndarray | None = None   # uint8 E4M3 bytes [M, K] (W4A8)
+    expert_ids: np.ndarray | None = None  # int32 [T, k] top-k routing (MoE layer)
     gA: float = 1.0                   # FP32 per-tensor scale of A_fp8
     # grouped
     E: int = 0
@@ -263,6 +264,20 @@ def grouped_w4a4(E: int = 8, tokens: int = 8192, N: int = 14336, K: int = 4096,
     W_e = [quantize_nvfp4_chunked(rngw, N, K, 0.02) for _ in range(E)]
     return Workload(f"grouped_w4a4_E{E}_T{M}_{N}x{K}", M, N, K, A=A, E=E, offsets=offsets,
                     W_e=W_e, notes="counts %s" % list(counts))
+
+
+def moe_layer(E: int = 8, tokens: int = 8192, N: int = 14336, K: int = 4096, seed_a: int = 0,
+              seed_w: int = 1, seed_route: int = 2) -> Workload:
+    """One MoE layer from BF16 tokens: X ~ N(0,1) [T,K] in token order (seed 0), top-1
+    Zipf(1.1) routing (seed 2), the grouped workload's expert weights (seed 1)."""
+    rng = np.random.Generator(np.random.PCG64(seed_a))
+    X = to_bf16_bits(rng.standard_normal((tokens, K), dtype=np.float32))
+    ids = zipf_routing(tokens, E, 1.1, seed_route).astype(np.int32).reshape(tokens, 1)
+    rngw = np.random.Generator(np.random.PCG64(seed_w))
+    W_e = [quantize_nvfp4_chunked(rngw, N, K, 0.02) for _ in range(E)]
+    return Workload(f"moe_layer_E{E}_T{tokens}_{N}x{K}", tokens, N, K, A_bf16=X, E=E, W_e=W_e,
+                    expert_ids=ids, notes="X bf16 N(0,1) seed %d, top-1 Zipf(1.1) seed %d, "
+                                          "W_e~N(0,0.02) seed %d" % (seed_a, seed_route, seed_w))
 
 
 def stack_experts(wl: Workload):
