@@ -29,7 +29,8 @@ __all__ = [
     "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
     "gemm_nvfp4_w4a4_packed", "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
     "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "nvfp4_fp4_fallback",
-    "nvfp4_node_exec", "moe_route", "moe_permute_rows", "moe_combine", "C_FUNCTIONS",
+    "nvfp4_node_exec", "moe_route", "moe_permute_rows", "moe_combine", "GroupedSchedule",
+    "C_FUNCTIONS",
 ]
 
 
@@ -101,6 +102,11 @@ C_FUNCTIONS = {
     "nvfp4_moe_route": (_I, [_P, _I, _I, _P, _P, _P, _P, _Z, _P]),
     "nvfp4_moe_permute_rows": (_I, [_P, _Z, _I, _I, _I, _P, _P, _P]),
     "nvfp4_moe_combine": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _P]),
+    "nvfp4_grouped_sched_bytes": (_Z, []),
+    "nvfp4_grouped_scale_layout_bytes_bound": (_Z, [_I, _I, _I]),
+    "nvfp4_grouped_schedule": (_I, [_P, _I, _I, _I, _I, _P, _F, _P, _P, _P]),
+    "nvfp4_pack_scales_grouped_sched": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "gemm_nvfp4_w4a4_grouped_packed_sched": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _P]),
     "nvfp4_quantize_bf16": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "nvfp4_quantize_bf16_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _P]),
 }
@@ -513,3 +519,56 @@ def moe_combine(Yg, dest, weights, T, k, out=None, stream=None):
     po = _dev_tensor(out, torch.bfloat16, (T, N), "out")
     _err(load_library().nvfp4_moe_combine(py, P, pd, pw, int(T), int(k), N, po, _stream_ptr(stream)))
     return out
+
+
+# --- grouped product planned on the device ------------------------------------------
+
+class GroupedSchedule:
+    """The grouped product's tile schedule planned on the device from device offsets.
+
+    sched = GroupedSchedule(offsets_dev, E, M, N, K, gW, gA=None or a 1-element CUDA
+    float32 tensor or a float).  Then pack(sA_plain) -> packed activation scales and
+    gemm(A, sA_packed, W, sW_packed) -> Y, with no host round trip."""
+
+    def __init__(self, offsets, E, M, N, K, gW, gA=1.0, stream=None):
+        import ctypes
+        torch = _torch()
+        self.E, self.M, self.N, self.K = int(E), int(M), int(N), int(K)
+        lib = load_library()
+        po = _dev_tensor(offsets, torch.int32, (self.E + 1,), "offsets")
+        self.buf = torch.empty(int(lib.nvfp4_grouped_sched_bytes()), dtype=torch.uint8,
+                               device=offsets.device)
+        gws = (ctypes.c_float * self.E)(*[float(x) for x in gW])
+        ga_dev, ga = None, 1.0
+        if isinstance(gA, torch.Tensor):
+            ga_dev = _dev_tensor(gA.reshape(-1)[:1], torch.float32, (1,), "gA")
+        else:
+            ga = float(gA)
+        _err(lib.nvfp4_grouped_schedule(po, self.E, self.M, self.N, self.K, ga_dev, ga,
+                                        ctypes.cast(gws, ctypes.c_void_p), self.buf.data_ptr(),
+                                        _stream_ptr(stream)))
+
+    def pack(self, s_plain, out=None, stream=None):
+        torch = _torch()
+        ps = _dev_tensor(s_plain, torch.uint8, (self.M, self.K // 16), "s_plain")
+        n = int(load_library().nvfp4_grouped_scale_layout_bytes_bound(self.M, self.E, self.K))
+        if out is None:
+            out = torch.empty(max(n, 16), dtype=torch.uint8, device=s_plain.device)
+        if out.dtype != torch.uint8 or not out.is_cuda or out.numel() < n or not out.is_contiguous():
+            raise ValueError(f"out must be a contiguous CUDA uint8 tensor of >= {n} bytes")
+        _err(load_library().nvfp4_pack_scales_grouped_sched(ps, self.M, self.E, self.K,
+                                                            self.buf.data_ptr(), out.data_ptr(),
+                                                            _stream_ptr(stream)))
+        return out
+
+    def gemm(self, A, sA_packed, W, sW_packed, out=None, stream=None):
+        torch = _torch()
+        pa = _dev_tensor(A, torch.uint8, (self.M, self.K // 2), "A")
+        pw = _dev_tensor(W, torch.uint8, (self.E, self.N, self.K // 2), "W")
+        if out is None:
+            out = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=A.device)
+        py = _dev_tensor(out, torch.bfloat16, (self.M, self.N), "out")
+        _err(load_library().gemm_nvfp4_w4a4_grouped_packed_sched(
+            pa, sA_packed.data_ptr(), pw, sW_packed.data_ptr(), self.buf.data_ptr(), self.E,
+            self.M, py, self.N, self.K, _stream_ptr(stream)))
+        return out

@@ -27,6 +27,7 @@
 
 #include "ptx.cuh"
 #include "w4a4_pair_kernel.cuh"
+#include "pack_scales_kernel.cuh"
 
 namespace nvfp4 {
 namespace grouped_pair {
@@ -146,7 +147,12 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
                     const __grid_constant__ CUtensorMap tmSW1,  // packed sW, box (128,16,1)
                     const __grid_constant__ CUtensorMap tmY,    // Y bf16 [M][N], box 64 x 32, 128B swizzle
                     int tma_out,                                // tmY is valid (N % 8 == 0)
-                    const __grid_constant__ Params p, __nv_bfloat16* __restrict__ Y) {
+                    const __grid_constant__ Params p_param,
+                    const Params* __restrict__ p_dev,           // schedule in device memory, or null
+                    __nv_bfloat16* __restrict__ Y) {
+    // the tile schedule: kernel parameters planned on the host, or device memory
+    // written by grouped_schedule_kernel from device-resident expert offsets
+    const Params& p = p_dev ? *p_dev : p_param;
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~uintptr_t(1023));
@@ -337,6 +343,45 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
     cluster_sync();
     tc_fence_after();
     if (warp == 1) tmem_dealloc_pair(tmem, TMEM_COLS);
+}
+
+// The tile schedule from device-resident expert offsets (one thread; E <= 256):
+// what the host-planned entry point computes, written to device memory, plus
+// the grouped packing map of the activations' scales.  Offsets that are not a
+// non-decreasing run from 0 to M give an empty schedule and a device error bit.
+constexpr int BAD_OFFSETS = 0x20000;
+struct GwArray {
+    float v[MAX_EXPERTS];
+};
+
+__global__ void grouped_schedule_kernel(const int32_t* __restrict__ offsets, int E, int M, int N,
+                                        int K, const float* __restrict__ gA_dev, float gA_host,
+                                        const __grid_constant__ GwArray gw, Params* __restrict__ out,
+                                        pack::GroupedPack* __restrict__ pk) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    const float gA = gA_dev ? *gA_dev : gA_host;
+    bool ok = offsets[0] == 0 && offsets[E] == M;
+    for (int e = 0; e < E && ok; ++e) ok = offsets[e + 1] >= offsets[e];
+    out->E = E;
+    out->N = N;
+    out->K = K;
+    pk->groups_n = E;
+    int total = 0, blocks = 0;
+    for (int e = 0; e <= E; ++e) {
+        const int r = ok ? offsets[e] : 0;
+        out->tile_start[e] = total;
+        out->row_start[e] = r;
+        out->block_start[e] = blocks;
+        pk->row_start[e] = r;
+        pk->block_start[e] = blocks;
+        if (e < E) {
+            out->alpha[e] = gA * gw.v[e];
+            const int Me = ok ? offsets[e + 1] - offsets[e] : 0;
+            total += tiles_of_expert(Me, N);
+            blocks += (Me + 127) / 128;
+        }
+    }
+    if (!ok) atomicOr(&g_device_error, BAD_OFFSETS);
 }
 
 }  // namespace grouped_pair

@@ -360,6 +360,9 @@ nvfp4_status nvfp4_check_device_error(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
     if (v & 0xFF)
         return fail(NVFP4_ERR_DEVICE_TIMEOUT, "a kernel wait expired (role %d)", (v >> 8) & 0xFF);
+    if (v & nvfp4::grouped_pair::BAD_OFFSETS)
+        return fail(NVFP4_ERR_INVALID_ARG,
+                    "device expert offsets were not a non-decreasing run from 0 to M");
     return fail(NVFP4_ERR_INVALID_ARG, "a routed expert id was outside [0, E)");
 }
 
@@ -919,7 +922,7 @@ nvfp4_status nvfp4_pack_scales_grouped(const uint8_t* s_plain, const int32_t* of
     const dim3 grid((unsigned)blocks, (unsigned)((ksteps + pk::KCHUNK - 1) / pk::KCHUNK));
     if (grid.y > 65535) return fail(NVFP4_ERR_INVALID_ARG, "K too large for packing");
     pk::pack_scales_grouped_kernel<<<grid, pk::ROWS, 0, static_cast<cudaStream_t>(stream)>>>(
-        s_plain, s_packed, gp, K / 16, ksteps);
+        s_plain, s_packed, gp, nullptr, K / 16, ksteps);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "launching pack_scales_grouped_kernel");
     return ok();
@@ -994,7 +997,126 @@ nvfp4_status gemm_nvfp4_w4a4_grouped_packed(const uint8_t* A, const uint8_t* sA_
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, gp::grouped_pair_kernel, tmA, tmA64, tmW, tmSA, tmSW2,
-                                       tmSW1, tmY, tma_out, prm,
+                                       tmSW1, tmY, tma_out, prm, (const gp::Params*)nullptr,
+                                       reinterpret_cast<__nv_bfloat16*>(Y));
+    if (e != cudaSuccess) return cuda_fail(e, "launching grouped_pair_kernel");
+    return ok();
+}
+
+// ------------------------------------------------------------------------- grouped, device offsets
+size_t nvfp4_grouped_sched_bytes(void) {
+    return ((sizeof(nvfp4::grouped_pair::Params) + 255) / 256) * 256 +
+           ((sizeof(nvfp4::pack::GroupedPack) + 255) / 256) * 256;
+}
+
+size_t nvfp4_grouped_scale_layout_bytes_bound(int M, int E, int K) {
+    if (M < 0 || E < 1 || K < 64 || K % 64 != 0) return 0;
+    return ((size_t)(M + 127) / 128 + (size_t)E) * 128 * (size_t)(K / 16);
+}
+
+namespace {
+nvfp4::grouped_pair::Params* sched_params(void* sched) {
+    return static_cast<nvfp4::grouped_pair::Params*>(sched);
+}
+nvfp4::pack::GroupedPack* sched_pack(void* sched) {
+    return reinterpret_cast<nvfp4::pack::GroupedPack*>(
+        static_cast<uint8_t*>(sched) + ((sizeof(nvfp4::grouped_pair::Params) + 255) / 256) * 256);
+}
+}  // namespace
+
+nvfp4_status nvfp4_grouped_schedule(const int32_t* offsets_dev, int E, int M, int N, int K,
+                                    const float* gA_dev, float gA, const float* gW_host,
+                                    void* sched, void* stream) {
+    namespace gp = nvfp4::grouped_pair;
+    if (E < 1 || E > gp::MAX_EXPERTS)
+        return fail(NVFP4_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", gp::MAX_EXPERTS, E);
+    if (M < 0 || N < 1 || K < gp::BK || K % gp::BK != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "M >= 0, N >= 1 and K %% 256 == 0 required");
+    if (!offsets_dev || !gW_host || !sched) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(sched)) return fail(NVFP4_ERR_MISALIGNED, "the schedule buffer must be 16-byte aligned");
+    gp::GwArray gw;
+    memset(&gw, 0, sizeof(gw));
+    for (int e = 0; e < E; ++e) gw.v[e] = gW_host[e];
+    gp::grouped_schedule_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        offsets_dev, E, M, N, K, gA_dev, gA, gw, sched_params(sched), sched_pack(sched));
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "launching grouped_schedule_kernel");
+}
+
+nvfp4_status nvfp4_pack_scales_grouped_sched(const uint8_t* s_plain, int M, int E, int K,
+                                             const void* sched, uint8_t* s_packed, void* stream) {
+    namespace pk = nvfp4::pack;
+    if (M < 0 || E < 1 || E > pk::MAX_GROUPS)
+        return fail(NVFP4_ERR_INVALID_ARG, "M >= 0 and E in [1, %d] required", pk::MAX_GROUPS);
+    if (K < 64 || K % 64 != 0) return fail(NVFP4_ERR_INVALID_ARG, "packing needs K %% 64 == 0 (got %d)", K);
+    if (M == 0) return ok();
+    if (!s_plain || !s_packed || !sched) return fail(NVFP4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(s_plain) || !aligned16(s_packed))
+        return fail(NVFP4_ERR_MISALIGNED, "s_plain and s_packed must be 16-byte aligned");
+    pk::GroupedPack none;
+    memset(&none, 0, sizeof(none));
+    const int ksteps = K / 64;
+    const dim3 grid((unsigned)((M + 127) / 128 + E), (unsigned)((ksteps + pk::KCHUNK - 1) / pk::KCHUNK));
+    if (grid.y > 65535) return fail(NVFP4_ERR_INVALID_ARG, "K too large for packing");
+    pk::pack_scales_grouped_kernel<<<grid, pk::ROWS, 0, static_cast<cudaStream_t>(stream)>>>(
+        s_plain, s_packed, none, sched_pack(const_cast<void*>(sched)), K / 16, ksteps);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "launching pack_scales_grouped_kernel");
+}
+
+nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched(const uint8_t* A, const uint8_t* sA_packed,
+                                                  const uint8_t* W, const uint8_t* sW_packed,
+                                                  const void* sched, int E, int M, void* Y, int N,
+                                                  int K, void* stream) {
+    namespace gp = nvfp4::grouped_pair;
+    if (E < 1 || E > gp::MAX_EXPERTS)
+        return fail(NVFP4_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", gp::MAX_EXPERTS, E);
+    nvfp4_status st = check_w4a4_args(A, sA_packed, W, sW_packed, Y, M, N, K);
+    if (st != NVFP4_OK) return st;
+    if (K % gp::BK != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "the grouped path needs K %% 256 == 0 (got %d)", K);
+    if ((int64_t)E * N > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "E*N too large");
+    if (!sched) return fail(NVFP4_ERR_INVALID_ARG, "null schedule");
+    int dev;
+    DevInfo info;
+    if ((st = check_fp4_path(dev, info)) != NVFP4_OK) return st;
+    if (M == 0 || N == 0) return ok();
+    if (info.num_sms < 2) return fail(NVFP4_ERR_CUDA, "the pair kernel needs at least two SMs");
+    CUtensorMap tmA, tmA64, tmW, tmSA, tmSW2, tmSW1;
+    const uint64_t ks = (uint64_t)K / 64;
+    const uint64_t wblocks = (uint64_t)E * ((N + 127) / 128);
+    const uint64_t ablocks = (uint64_t)(M + 127) / 128 + (uint64_t)E;  // the packed sA bound
+    if ((st = make_map_u8(&tmA, A, (uint64_t)K / 2, (uint64_t)M, gp::BKB, gp::BM)) != NVFP4_OK) return st;
+    if ((st = make_map_u8(&tmA64, A, (uint64_t)K / 2, (uint64_t)M, gp::BKB, gp::SWAP_HALF)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_u8(&tmW, W, (uint64_t)K / 2, (uint64_t)E * N, gp::BKB, gp::BNH)) != NVFP4_OK)
+        return st;
+    if ((st = make_map_packed_sf(&tmSA, sA_packed, ablocks, ks, 1)) != NVFP4_OK) return st;
+    if ((st = make_map_packed_sf(&tmSW2, sW_packed, wblocks, ks, gp::NRB)) != NVFP4_OK) return st;
+    if ((st = make_map_packed_sf(&tmSW1, sW_packed, wblocks, ks, 1)) != NVFP4_OK) return st;
+    CUtensorMap tmY;
+    int tma_out = 0;
+    if ((st = make_map_out(&tmY, Y, (uint64_t)M, (uint64_t)N, tma_out)) != NVFP4_OK) return st;
+    if ((st = set_smem(gp::grouped_pair_kernel, gp::SMEM_BYTES, info, "grouped_pair_kernel")) != NVFP4_OK)
+        return st;
+    gp::Params none;
+    memset(&none, 0, sizeof(none));
+    // the tile count is on the device: one cluster per SM pair, idle clusters return
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (info.num_sms / 2));
+    cfg.blockDim = dim3(gp::NUM_THREADS);
+    cfg.dynamicSmemBytes = gp::SMEM_BYTES;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gp::grouped_pair_kernel, tmA, tmA64, tmW, tmSA, tmSW2,
+                                       tmSW1, tmY, tma_out, none,
+                                       (const gp::Params*)sched_params(const_cast<void*>(sched)),
                                        reinterpret_cast<__nv_bfloat16*>(Y));
     if (e != cudaSuccess) return cuda_fail(e, "launching grouped_pair_kernel");
     return ok();

@@ -67,10 +67,16 @@ struct GroupedPack {
     int block_start[MAX_GROUPS + 1];
 };
 
+// The map comes from the kernel parameters, or, when gp_dev is not null, from
+// device memory (written by the grouped schedule kernel); then the grid is an
+// upper bound and CTAs past the last block return.
 __global__ void __launch_bounds__(ROWS)
 pack_scales_grouped_kernel(const uint8_t* __restrict__ s, uint8_t* __restrict__ out,
-                           const __grid_constant__ GroupedPack gp, int groups, int ksteps) {
+                           const __grid_constant__ GroupedPack gp_param,
+                           const GroupedPack* __restrict__ gp_dev, int groups, int ksteps) {
+    const GroupedPack& gp = gp_dev ? *gp_dev : gp_param;
     const int b = blockIdx.x;
+    if (b >= gp.block_start[gp.groups_n]) return;
     int lo = 0, hi = gp.groups_n;  // block_start[lo] <= b < block_start[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;

@@ -370,6 +370,48 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_packed(const uint8_t* A, const ui
                                                       const int32_t* offsets_host, int E,
                                                       void* Y_bf16, int N, int K, void* stream);
 
+/* ---- grouped product with device-resident expert offsets -----------------
+ * The grouped entry points above plan their tiles on the host from host
+ * offsets.  These take offsets[E+1] in device memory (for example from
+ * nvfp4_moe_route), so a whole MoE layer runs with no host round trip and can
+ * be captured in a CUDA graph: nvfp4_grouped_schedule plans on the device into
+ * a small caller buffer, which the packing and the product then read.  Same
+ * operation, layouts and rounding as gemm_nvfp4_w4a4_grouped_packed. */
+
+/* Bytes of the schedule buffer (device memory, 16-byte aligned, caller-owned). */
+NVFP4_API size_t nvfp4_grouped_sched_bytes(void);
+
+/* Upper bound of the grouped packed layout of M rows in E groups, whatever the
+ * offsets: (ceil(M/128) + E) * 128 * K/16 bytes (0 for bad sizes).  The packed
+ * activation scales of the scheduled path need a buffer of this size. */
+NVFP4_API size_t nvfp4_grouped_scale_layout_bytes_bound(int M, int E, int K);
+
+/* One thread on the device reads offsets_dev [E+1] (int32, offsets[0] = 0,
+ * non-decreasing, offsets[E] = M) and writes the tile schedule, alpha_e =
+ * gA*gW[e] (gA from *gA_dev when gA_dev is not null, else the host value gA;
+ * gW_host [E] host floats read during the call) and the packing map into
+ * `sched`.  Offsets that break those rules give an empty schedule (the
+ * products below then write nothing) and make the next
+ * nvfp4_check_device_error return NVFP4_ERR_INVALID_ARG.  E in [1, 256]; N >= 1;
+ * K % 256 == 0. */
+NVFP4_API nvfp4_status nvfp4_grouped_schedule(const int32_t* offsets_dev, int E, int M, int N, int K,
+                                              const float* gA_dev, float gA, const float* gW_host,
+                                              void* sched, void* stream);
+
+/* nvfp4_pack_scales_grouped with the groups of a schedule: s_plain [M][K/16] ->
+ * s_packed (nvfp4_grouped_scale_layout_bytes_bound(M, E, K) bytes). */
+NVFP4_API nvfp4_status nvfp4_pack_scales_grouped_sched(const uint8_t* s_plain, int M, int E, int K,
+                                                       const void* sched, uint8_t* s_packed,
+                                                       void* stream);
+
+/* gemm_nvfp4_w4a4_grouped_packed with the tiles and alphas of a schedule: A
+ * [M][K/2] grouped by expert, sA_packed from nvfp4_pack_scales_grouped_sched, W
+ * [E][N][K/2] and sW_packed as for the host-planned entry, Y [M][N]. */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched(const uint8_t* A, const uint8_t* sA_packed,
+                                                            const uint8_t* W, const uint8_t* sW_packed,
+                                                            const void* sched, int E, int M, void* Y_bf16,
+                                                            int N, int K, void* stream);
+
 /* ---- diagnostics ----------------------------------------------------------- */
 
 /* Thread-local text of the last error returned on this host thread ("" if none). */
@@ -378,7 +420,8 @@ NVFP4_API const char* nvfp4_last_error(void);
 /* Synchronizes `stream`, then reads and clears the device error word that a
  * kernel sets when one of its bounded waits expires.  NVFP4_OK if clear,
  * NVFP4_ERR_DEVICE_TIMEOUT if a wait expired, NVFP4_ERR_INVALID_ARG if the only
- * record is an out-of-range expert id seen by nvfp4_moe_route, NVFP4_ERR_CUDA if
+ * records are bad data seen on the device (an out-of-range expert id in
+ * nvfp4_moe_route, bad offsets in nvfp4_grouped_schedule), NVFP4_ERR_CUDA if
  * synchronization failed. */
 NVFP4_API nvfp4_status nvfp4_check_device_error(void* stream);
 

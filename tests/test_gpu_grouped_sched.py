@@ -1,0 +1,144 @@
+"""The grouped product planned on the device from device-resident expert offsets:
+the same bytes as the host-planned entry (same tiles, same alphas), parity with the
+oracle, bad offsets reported, and a whole MoE layer captured in one CUDA graph."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import block_scaled_precision_nvfp4_b200 as nv
+from block_scaled_precision_nvfp4_b200 import workloads as wl
+
+from parity import bf16_to_f64, check
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _random_grouped(counts, N, K, seed):
+    rng = np.random.default_rng(seed)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    A = wl.uniform_operand(rng, int(off[-1]), K)
+    Ws = [wl.uniform_operand(rng, N, K) for _ in counts]
+    Wc = np.stack([w.codes for w in Ws]); Wsc = np.stack([w.scales for w in Ws])
+    gW = rng.choice([0.25, 0.5, 1.0, 2.0], len(counts))
+    return A, Wc, Wsc, gW, off
+
+
+COUNTS = [([1, 8, 17, 64, 127, 128], 520, 512), ([0, 130, 0, 1, 256, 300], 264, 256),
+          ([127, 128, 129, 383, 384, 385], 136, 768), ([16], 1000, 1024), ([40] * 20, 384, 256),
+          ([5, 300, 129, 64], 100, 256), ([0, 0, 0], 256, 256)]
+
+
+@pytest.mark.parametrize("counts,N,K", COUNTS)
+def test_device_schedule_equals_host_plan(counts, N, K):
+    A, Wc, Ws, gW, off = _random_grouped(counts, N, K, sum(counts) * 3 + N + K)
+    E, M = len(counts), int(off[-1])
+    sw = nv.nvfp4_pack_scales_grouped(_dev(Ws.reshape(E * N, K // 16)),
+                                      [e * N for e in range(E + 1)], K)
+    sched = nv.GroupedSchedule(_dev(off.astype(np.int32)), E, M, N, K, gW, gA=1.5)
+    sa_d = sched.pack(_dev(A.scales))
+    y_d = sched.gemm(_dev(A.codes), sa_d, _dev(Wc), sw)
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    if M == 0:
+        assert y_d.numel() == 0
+        return
+    sa_h = nv.nvfp4_pack_scales_grouped(_dev(A.scales), list(off), K)
+    y_h = nv.gemm_nvfp4_w4a4_grouped_packed(_dev(A.codes), sa_h, 1.5, _dev(Wc), sw, list(gW),
+                                            list(off))
+    torch.cuda.synchronize()
+    n = nv.nvfp4_grouped_scale_layout_bytes(list(off), K)
+    assert torch.equal(sa_d[:n], sa_h[:n])
+    assert torch.equal(y_d.view(torch.int16), y_h.view(torch.int16))
+    ref = oracle.gemm_grouped_w4a4(A.codes, A.scales, 1.5, Wc, Ws, gW, off, N, K)
+    check(bf16_to_f64(y_d), ref, f"grouped sched {counts}")
+
+
+def test_device_gA_equals_host_gA():
+    A, Wc, Ws, gW, off = _random_grouped([100, 0, 257], 256, 512, 5)
+    E, N, K, M = 3, 256, 512, int(off[-1])
+    sw = nv.nvfp4_pack_scales_grouped(_dev(Ws.reshape(E * N, K // 16)),
+                                      [e * N for e in range(E + 1)], K)
+    ga = torch.tensor([0.375], dtype=torch.float32, device="cuda")
+    ys = []
+    for g in (ga, 0.375):
+        s = nv.GroupedSchedule(_dev(off.astype(np.int32)), E, M, N, K, gW, gA=g)
+        ys.append(s.gemm(_dev(A.codes), s.pack(_dev(A.scales)), _dev(Wc), sw))
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0].view(torch.int16), ys[1].view(torch.int16))
+
+
+def test_bad_device_offsets_are_reported_and_write_nothing():
+    A, Wc, Ws, gW, off = _random_grouped([64, 64], 256, 256, 9)
+    E, N, K, M = 2, 256, 256, 128
+    sw = nv.nvfp4_pack_scales_grouped(_dev(Ws.reshape(E * N, K // 16)), [0, N, 2 * N], K)
+    bad = torch.tensor([0, 100, 90], dtype=torch.int32, device="cuda")   # decreasing, wrong end
+    s = nv.GroupedSchedule(bad, E, M, N, K, gW)
+    y = torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    s.gemm(_dev(A.codes), s.pack(_dev(A.scales)), _dev(Wc), sw, out=y)
+    with pytest.raises(nv.NvFp4Error) as e:
+        nv.nvfp4_check_device_error()
+    assert e.value.status == nv.Status.INVALID_ARG
+    assert bool((y.float() == 7.0).all())
+
+
+def test_whole_moe_layer_in_one_cuda_graph():
+    """quantise -> route -> permute -> schedule -> pack -> grouped W4A4 -> combine,
+    captured once and replayed, equals the eager layer bit for bit."""
+    rng = np.random.default_rng(21)
+    T, E, N, K = 700, 4, 384, 512
+    x = torch.from_numpy(rng.standard_normal((T, K)).astype(np.float32)).to(torch.bfloat16).cuda()
+    ids = torch.from_numpy(rng.integers(0, E, size=(T, 1)).astype(np.int32)).cuda()
+    w = torch.ones((T, 1), dtype=torch.float32, device="cuda")
+    experts = [wl.quantize_nvfp4(rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02))
+               for _ in range(E)]
+    Wc = _dev(np.stack([e.codes for e in experts]))
+    sw = nv.nvfp4_pack_scales_grouped(_dev(np.stack([e.scales for e in experts]).reshape(E * N, -1)),
+                                      [e * N for e in range(E + 1)], K)
+    gws = [e.g for e in experts]
+    lib = nv.load_library()
+    route_ws = torch.empty(lib.nvfp4_moe_route_workspace_bytes(T, E), dtype=torch.uint8, device="cuda")
+    q_ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    bufs = dict(codes=torch.empty((T, K // 2), dtype=torch.uint8, device="cuda"),
+                scales=torch.empty((T, K // 16), dtype=torch.uint8, device="cuda"),
+                g=torch.empty(4, dtype=torch.float32, device="cuda"),
+                gc=torch.empty((T, K // 2), dtype=torch.uint8, device="cuda"),
+                gs=torch.empty((T, K // 16), dtype=torch.uint8, device="cuda"),
+                sa=torch.empty(lib.nvfp4_grouped_scale_layout_bytes_bound(T, E, K), dtype=torch.uint8,
+                               device="cuda"),
+                yg=torch.empty((T, N), dtype=torch.bfloat16, device="cuda"),
+                y=torch.empty((T, N), dtype=torch.bfloat16, device="cuda"))
+
+    def layer(s):
+        b = bufs
+        nv.nvfp4_quantize_bf16(x, plain=True, packed=False, workspace=q_ws, stream=s,
+                               out=(b["codes"], b["scales"], None, b["g"]))
+        off, dest, src = nv.moe_route(ids, E, workspace=route_ws, stream=s)
+        nv.moe_permute_rows(b["codes"], src, 1, out=b["gc"], stream=s)
+        nv.moe_permute_rows(b["scales"], src, 1, out=b["gs"], stream=s)
+        sched = nv.GroupedSchedule(off, E, T, N, K, gws, gA=b["g"][:1], stream=s)
+        sched.pack(b["gs"], out=b["sa"], stream=s)
+        sched.gemm(b["gc"], b["sa"], Wc, sw, out=b["yg"], stream=s)
+        nv.moe_combine(b["yg"], dest, w, T, 1, out=b["y"], stream=s)
+        return sched, off, dest, src
+
+    cur = torch.cuda.current_stream()
+    keep = layer(cur)
+    torch.cuda.synchronize()
+    eager = bufs["y"].clone()
+    bufs["y"].zero_()
+    s = torch.cuda.Stream()
+    s.wait_stream(cur)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        keep2 = layer(s)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    assert torch.equal(bufs["y"].view(torch.int16), eager.view(torch.int16))
+    del g
