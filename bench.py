@@ -426,34 +426,35 @@ def run_ours(args):
                                dtype=torch.uint8, device=dev)
         gc_b = torch.empty_like(codes_b)
         gs_b = torch.empty_like(scales_b)
-        sa_b = torch.empty(nv.nvfp4_grouped_scale_layout_bytes([0] * E + [M], K) + 128 * (K // 16) * E,
-                           dtype=torch.uint8, device=dev)
         Yg_b = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ones = torch.ones((M, 1), dtype=torch.float32, device=dev)
 
-        def step(stages=None):
+        sa_b = torch.empty(nv.load_library().nvfp4_grouped_scale_layout_bytes_bound(M, E, K),
+                           dtype=torch.uint8, device=dev)
+
+        def step(stages=None, s=None):
+            # the whole layer on the device: the grouped product is planned from the
+            # route's device offsets and the quantiser's device gA, so no host round trip
+            s = s or stream
+
             def mark(i):
                 if stages is not None:
-                    stages[i].record(stream)
+                    stages[i].record(s)
             mark(0)
             nv.nvfp4_quantize_bf16(dv[0].view(torch.bfloat16), plain=True, packed=False,
-                                   workspace=q_ws, stream=stream, out=(codes_b, scales_b, None, g_b))
+                                   workspace=q_ws, stream=s, out=(codes_b, scales_b, None, g_b))
             mark(1)
-            off, dest, src = nv.moe_route(dv[1], E, workspace=route_ws, stream=stream)
+            off, dest, src = nv.moe_route(dv[1], E, workspace=route_ws, stream=s)
             mark(2)
-            nv.moe_permute_rows(codes_b, src, 1, out=gc_b, stream=stream)
-            nv.moe_permute_rows(scales_b, src, 1, out=gs_b, stream=stream)
+            nv.moe_permute_rows(codes_b, src, 1, out=gc_b, stream=s)
+            nv.moe_permute_rows(scales_b, src, 1, out=gs_b, stream=s)
             mark(3)
-            # the grouped product plans its tiles on the host: offsets and gA come back
-            host_vals = torch.cat([off.to(torch.float64), g_b[:1].to(torch.float64)]).cpu()
-            offsets = [int(x) for x in host_vals[:E + 1]]
-            gA = float(host_vals[E + 1])
-            nv.nvfp4_pack_scales_grouped(gs_b, offsets, K, out=sa_b, stream=stream)
+            sched = nv.GroupedSchedule(off, E, M, N, K, gws, gA=g_b[:1], stream=s)
+            sched.pack(gs_b, out=sa_b, stream=s)
             mark(4)
-            nv.gemm_nvfp4_w4a4_grouped_packed(gc_b, sa_b, gA, Wc_d, sw_packed, gws, offsets,
-                                              out=Yg_b, stream=stream)
+            sched.gemm(gc_b, sa_b, Wc_d, sw_packed, out=Yg_b, stream=s)
             mark(5)
-            nv.moe_combine(Yg_b, dest, ones, M, 1, out=Y, stream=stream)
+            nv.moe_combine(Yg_b, dest, ones, M, 1, out=Y, stream=s)
             mark(6)
     elif path == "w4a8":
         def step():
@@ -479,7 +480,7 @@ def run_ours(args):
         def plain_step():
             nv.gemm_nvfp4_w4a4(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
     launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2, "grouped": 2, "quantize": 2,
-                         "moe": 10}.get(path, 1)
+                         "moe": 11}.get(path, 1)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -487,12 +488,12 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     nv.nvfp4_check_device_error(stream)
 
-    # The two-launch steps (pack the activations' scales, then the product) are also
-    # captured once in a CUDA graph; its replay times the same two kernels without the
-    # host launch gap between them, and gives `value`.  The eager loop below still
-    # times the product alone between events.
+    # The multi-launch steps (pack the activations' scales, then the product; the whole
+    # MoE layer) are also captured once in a CUDA graph; its replay times the same
+    # kernels without the host launch gaps between them, and gives `value`.  The eager
+    # loop below still times the product (and the MoE stages) between events.
     graph, launch = None, "eager"
-    if path in ("w4a4", "grouped") and not args.no_graph:
+    if path in ("w4a4", "grouped", "moe") and not args.no_graph:
         try:
             gstream = torch.cuda.Stream(dev)
             gstream.wait_stream(stream)
@@ -650,7 +651,7 @@ def run_ours(args):
                  "plain_scale_entry_ms": statistics.median(plain),
                  "plain_scale_entry_tflops": flops / (statistics.median(plain) * 1e-3) / 1e12}
     if stage_ev is not None:
-        names = ["quantize", "route", "permute", "offsets_to_host_and_pack", "grouped_gemm", "combine"]
+        names = ["quantize", "route", "permute", "schedule_and_pack", "grouped_gemm", "combine"]
         med = {n: statistics.median(ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev) * 1e3
                for j, n in enumerate(names)}
         kern_s = med["grouped_gemm"] * 1e-6
