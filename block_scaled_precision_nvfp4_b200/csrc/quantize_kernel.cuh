@@ -71,10 +71,10 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(b | (b << 8))));
     return __half2float(__ushort_as_half((uint16_t)(h2 & 0xFFFFu)));
 }
-// eight magnitudes |t0| .. |t7| -> eight E2M1 magnitude codes, packed with
-// element 2j in the low nibble of byte j (cvt puts its first operand in the high
-// nibble)
-__device__ __forceinline__ uint32_t e2m1x8_mag(const float (&t)[8]) {
+// eight values t0 .. t7 -> eight signed E2M1 codes (the sign of t kept, -0 and
+// values that round to zero included), packed with element 2j in the low nibble
+// of byte j (cvt puts its first operand in the high nibble)
+__device__ __forceinline__ uint32_t e2m1x8(const float (&t)[8]) {
     uint32_t r;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -83,8 +83,7 @@ __device__ __forceinline__ uint32_t e2m1x8_mag(const float (&t)[8]) {
         "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
         "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
         : "=r"(r)
-        : "f"(fabsf(t[0])), "f"(fabsf(t[1])), "f"(fabsf(t[2])), "f"(fabsf(t[3])),
-          "f"(fabsf(t[4])), "f"(fabsf(t[5])), "f"(fabsf(t[6])), "f"(fabsf(t[7])));
+        : "f"(t[0]), "f"(t[1]), "f"(t[2]), "f"(t[3]), "f"(t[4]), "f"(t[5]), "f"(t[6]), "f"(t[7]));
     return r;
 }
 
@@ -132,16 +131,27 @@ quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
         const float den = __fmul_rn(e4m3_value(sb), g);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         float t[8];
-        uint32_t sgn = 0u;
+        // t = x / den, correctly rounded.  The divisor is shared by the group, so its
+        // correctly rounded reciprocal y is taken once and each quotient is finished by
+        // Markstein's correction (q = RN(x*y), r = x - den*q exactly by FMA,
+        // t = RN(q + r*y)), which gives RN(x/den) when no step under- or overflows:
+        // true for den in [2^-60, 2^60] (|t| stays below 7 by the choice of s).  Other
+        // groups, and den == 0, keep the plain division.
+        const bool fast = den >= 0x1p-60f && den <= 0x1p60f;
+        const float y = fast ? __frcp_rn(den) : 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             // element e is half (e & 1) of word e >> 1
             const uint32_t h = (e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16);
             const float xe = __uint_as_float(h);
-            t[e] = den > 0.f ? __fdiv_rn(xe, den) : xe * 0.0f;
-            sgn |= (__float_as_uint(t[e]) >> 31) << (4 * e + 3);
+            if (fast) {
+                const float q = __fmul_rn(xe, y);
+                t[e] = __fmaf_rn(__fmaf_rn(-q, den, xe), y, q);
+            } else {
+                t[e] = den > 0.f ? __fdiv_rn(xe, den) : xe * 0.0f;
+            }
         }
-        const uint32_t out = e2m1x8_mag(t) | sgn;
+        const uint32_t out = e2m1x8(t);
         if (ok) *reinterpret_cast<uint32_t*>(codes + (size_t)row * (K / 2) + col / 2) = out;
         // the group's scale byte: lane 2j holds group j; gather four groups (one K = 64
         // step) into one word in shared memory

@@ -138,3 +138,21 @@ def test_argument_errors():
     with pytest.raises(nv.NvFp4Error) as e:
         nv.nvfp4_quantize_bf16(x, packed=True)
     assert e.value.status == nv.Status.INVALID_ARG
+
+
+@pytest.mark.parametrize("dist", ["normal", "uniform", "cauchy", "wide"])
+def test_every_element_bit_exact_over_distributions(dist):
+    """8.4M elements compared one by one: the division by each group's s*g is the
+    correctly rounded FP32 quotient, so every code equals the oracle's."""
+    rng = np.random.default_rng({"normal": 1, "uniform": 2, "cauchy": 3, "wide": 4}[dist])
+    rows, K = 1024, 8192
+    if dist == "normal":
+        x = rng.standard_normal((rows, K)).astype(np.float32)
+    elif dist == "uniform":
+        x = rng.uniform(-3, 3, (rows, K)).astype(np.float32)
+    elif dist == "cauchy":
+        x = np.clip(rng.standard_cauchy((rows, K)), -1e30, 1e30).astype(np.float32)
+    else:   # blocks spread over 2^-100 .. 2^100
+        x = (rng.standard_normal((rows, K)) *
+             np.exp2(rng.integers(-100, 100, size=(rows, K // 16))).repeat(16, axis=1)).astype(np.float32)
+    _expect_equal(_bits(x), K)
