@@ -71,6 +71,18 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(b | (b << 8))));
     return __half2float(__ushort_as_half((uint16_t)(h2 & 0xFFFFu)));
 }
+// two FP32 lanes at once: d = RN(a*b), d = RN(a*b + c) per lane
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // eight values t0 .. t7 -> eight signed E2M1 codes (the sign of t kept, -0 and
 // values that round to zero included), packed with element 2j in the low nibble
 // of byte j (cvt puts its first operand in the high nibble)
@@ -138,16 +150,25 @@ quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
         // true for den in [2^-60, 2^60] (|t| stays below 7 by the choice of s).  Other
         // groups, and den == 0, keep the plain division.
         const bool fast = den >= 0x1p-60f && den <= 0x1p60f;
-        const float y = fast ? __frcp_rn(den) : 0.f;
+        if (fast) {
+            // both halves of a word at once (packed f32x2 lanes, each one IEEE RN op)
+            const float y = __frcp_rn(den);
+            const uint64_t y2 = ((uint64_t)__float_as_uint(y) << 32) | __float_as_uint(y);
+            const uint64_t nd2 = ((uint64_t)__float_as_uint(-den) << 32) | __float_as_uint(-den);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            // element e is half (e & 1) of word e >> 1
-            const uint32_t h = (e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16);
-            const float xe = __uint_as_float(h);
-            if (fast) {
-                const float q = __fmul_rn(xe, y);
-                t[e] = __fmaf_rn(__fmaf_rn(-q, den, xe), y, q);
-            } else {
+            for (int j = 0; j < 4; ++j) {
+                const uint64_t x2 = ((uint64_t)(w[j] & 0xFFFF0000u) << 32) | (uint64_t)(w[j] << 16);
+                const uint64_t q2 = mul_f32x2(x2, y2);
+                const uint64_t t2 = fma_f32x2(fma_f32x2(q2, nd2, x2), y2, q2);
+                t[2 * j] = __uint_as_float((uint32_t)t2);
+                t[2 * j + 1] = __uint_as_float((uint32_t)(t2 >> 32));
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                // element e is half (e & 1) of word e >> 1
+                const uint32_t h = (e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16);
+                const float xe = __uint_as_float(h);
                 t[e] = den > 0.f ? __fdiv_rn(xe, den) : xe * 0.0f;
             }
         }
