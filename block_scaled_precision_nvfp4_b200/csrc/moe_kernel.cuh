@@ -25,6 +25,27 @@ constexpr int ROUTE_WARPS = ROUTE_THREADS / 32;
 constexpr int MAX_CHUNKS = 128;              // route chunks (one CTA each) at most
 constexpr int BAD_EXPERT_ID = 0x10000;       // device error word bit: an id outside [0, E)
 
+// wcnt[w][x] (pairs of warp w for expert x in this sub-chunk) -> run[x] plus the
+// pairs of expert x in warps before w; run[x] advances by the sub-chunk's total.
+// Warp v takes experts v, v + 32, ...; its lanes scan the 32 warps' counts.
+__device__ __forceinline__ void prefix_over_warps(int32_t (&wcnt)[ROUTE_WARPS][MAX_EXPERTS],
+                                                  int32_t* run, int E) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int x = warp; x < E; x += ROUTE_WARPS) {
+        const int32_t c = wcnt[lane][x];
+        int32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int32_t base = run[x];
+        wcnt[lane][x] = base + incl - c;
+        __syncwarp();
+        if (lane == 31) run[x] = base + incl;
+    }
+}
+
 // Pass 1: counts[c][e] = pairs of chunk c routed to expert e.  Chunk c is
 // pairs [c*chunk, min((c+1)*chunk, P)).  An id outside [0, E) is left out of
 // every expert and recorded in the device error word.
@@ -105,15 +126,7 @@ route_rank_kernel(const int32_t* __restrict__ ids, int P, int E, int chunk,
         if (e >= 0 && lrank == 0) wcnt[warp][e] = __popc(peers);
         __syncthreads();
         // exclusive prefix over warps, per expert; then advance the running counts
-        for (int x = threadIdx.x; x < E; x += ROUTE_THREADS) {
-            int32_t r = run[x];
-            for (int w = 0; w < ROUTE_WARPS; ++w) {
-                const int32_t c = wcnt[w][x];
-                wcnt[w][x] = r;
-                r += c;
-            }
-            run[x] = r;
-        }
+        prefix_over_warps(wcnt, run, E);
         __syncthreads();
         if (e >= 0) {
             const int32_t d = wcnt[warp][e] + lrank;
@@ -121,6 +134,66 @@ route_rank_kernel(const int32_t* __restrict__ ids, int P, int E, int chunk,
             src[d] = p;
         }
         __syncthreads();
+    }
+}
+
+// The three passes in one CTA, for up to SMALL_PAIRS pairs (one launch, no memsets):
+// histogram, scan, then ranks by sub-chunks of 1024 pairs in order.  Pairs with an
+// out-of-range id get dest = -1; grouped rows past the last placed one get src = -1.
+constexpr int SMALL_PAIRS = 65536;
+
+__global__ void __launch_bounds__(ROUTE_THREADS)
+route_small_kernel(const int32_t* __restrict__ ids, int P, int E, int32_t* __restrict__ offsets,
+                   int32_t* __restrict__ dest, int32_t* __restrict__ src) {
+    __shared__ int32_t run[MAX_EXPERTS];
+    __shared__ int32_t wcnt[ROUTE_WARPS][MAX_EXPERTS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < E; e += ROUTE_THREADS) run[e] = 0;
+    __syncthreads();
+    for (int p0 = 0; p0 < P; p0 += ROUTE_THREADS) {  // whole warps: the match needs all lanes
+        const int p = p0 + threadIdx.x;
+        int e = p < P ? ids[p] : -1;
+        if (p < P && (e < 0 || e >= E)) {
+            atomicOr(&g_device_error, BAD_EXPERT_ID);
+            dest[p] = -1;
+        }
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);  // one atomic per expert per warp
+        if (e >= 0 && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&run[e], __popc(peers));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {  // exclusive scan over experts, in expert order
+        int32_t acc = 0;
+        for (int e = 0; e < E; ++e) {
+            const int32_t c = run[e];
+            run[e] = acc;
+            offsets[e] = acc;
+            acc += c;
+        }
+        offsets[E] = acc;
+        wcnt[0][0] = acc;  // placed pairs, read below before the first sub-chunk reset
+    }
+    __syncthreads();
+    const int placed = wcnt[0][0];
+    for (int r = placed + threadIdx.x; r < P; r += ROUTE_THREADS) src[r] = -1;
+    for (int s0 = 0; s0 < P; s0 += ROUTE_THREADS) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < ROUTE_WARPS * E; i += ROUTE_THREADS) wcnt[i / E][i % E] = 0;
+        __syncthreads();
+        const int p = s0 + threadIdx.x;
+        int e = p < P ? ids[p] : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int lrank = __popc(peers & ((1u << lane) - 1u));
+        if (e >= 0 && lrank == 0) wcnt[warp][e] = __popc(peers);
+        __syncthreads();
+        prefix_over_warps(wcnt, run, E);
+        __syncthreads();
+        if (e >= 0) {
+            const int32_t d = wcnt[warp][e] + lrank;
+            dest[p] = d;
+            src[d] = p;
+        }
     }
 }
 

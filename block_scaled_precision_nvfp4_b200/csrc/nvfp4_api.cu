@@ -706,6 +706,12 @@ nvfp4_status nvfp4_moe_route(const int32_t* expert_ids, int num_pairs, int E, in
         e = cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s);
         return e == cudaSuccess ? ok() : cuda_fail(e, "clearing the expert offsets");
     }
+    if (num_pairs <= mo::SMALL_PAIRS) {  // one CTA does all three passes
+        mo::route_small_kernel<<<1, mo::ROUTE_THREADS, 0, s>>>(expert_ids, num_pairs, E, offsets, dest,
+                                                               src);
+        e = cudaGetLastError();
+        return e == cudaSuccess ? ok() : cuda_fail(e, "launching route_small_kernel");
+    }
     // pairs with an out-of-range id are placed nowhere: their dest stays -1, and rows
     // no pair lands on keep src = -1
     if ((e = cudaMemsetAsync(dest, 0xFF, (size_t)num_pairs * sizeof(int32_t), s)) != cudaSuccess ||

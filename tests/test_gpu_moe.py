@@ -22,8 +22,10 @@ def _ids(rng, T, k, E, zipf=None):
     return rng.choice(E, size=(T, k), p=p / p.sum()).astype(np.int32)
 
 
+# up to 65536 pairs one CTA routes; beyond that, chunked histograms, a scan and ranks
 CASES = [(1, 1, 1, None), (7, 1, 4, None), (1000, 2, 64, None), (8192, 1, 8, 1.1),
-         (5000, 4, 256, None), (3000, 2, 16, 2.5), (2049, 3, 5, None)]
+         (5000, 4, 256, None), (3000, 2, 16, 2.5), (2049, 3, 5, None), (16384, 4, 8, None),
+         (40000, 2, 32, 1.1), (70001, 1, 256, None)]
 
 
 @pytest.mark.parametrize("T,k,E,zipf", CASES)
@@ -49,8 +51,11 @@ def test_route_empty_and_unused_experts():
     assert np.array_equal(off.cpu().numpy(), ro) and np.array_equal(dest.cpu().numpy(), rd)
 
 
-def test_route_bad_id_is_reported_and_left_out():
+@pytest.mark.parametrize("big", [False, True])
+def test_route_bad_id_is_reported_and_left_out(big):
     ids = np.array([0, 3, 9, 1, -2, 3], np.int32)
+    if big:   # past the one-CTA size
+        ids = np.concatenate([np.random.default_rng(0).integers(0, 4, 70000).astype(np.int32), ids])
     off, dest, src = nv.moe_route(torch.from_numpy(ids).cuda(), 4)
     with pytest.raises(nv.NvFp4Error) as e:
         nv.nvfp4_check_device_error()
