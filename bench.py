@@ -728,6 +728,8 @@ def run_ours(args):
         "value": value, "unit": "GB/s" if path == "quantize" else "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "step_ms_stats": {"median": statistics.median(per_step), "min": min(per_step),
+                          "p90": sorted(per_step)[min(len(per_step) - 1, int(0.9 * len(per_step)))]},
         "dtype": ("bf16 -> nvfp4 (fp32 scale arithmetic)" if path == "quantize" else
                   "bf16 x nvfp4(e2m1, e4m3 group scales) -> f32 accumulate -> bf16"
                   if path == "w4a16" else
