@@ -27,8 +27,9 @@
 //   warps 4-11  scale-apply + epilogue: per group, partial TMEM -> registers,
 //               acc += P * (sA*64)(sW*64) with packed f32x2 FMAs; at the end of
 //               a tile, x alpha, BF16 RNE, store.
-// This path is bound by the per-group FP32 scale-apply (ALU), not by the FP8
-// tensor pipe.  Requires K % 256 == 0 (TMA of the scale tiles).
+// Every 16-group's 128 x 128 FP32 partial leaves TMEM to be scaled, so the
+// per-group chain (MMA, commit, partial read-out, FP32 apply) sets the pace, not
+// the FP8 tensor pipe.  Requires K % 256 == 0 (TMA of the scale tiles).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>

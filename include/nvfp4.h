@@ -261,9 +261,11 @@ NVFP4_API nvfp4_status gemm_nvfp4_via_fp8(const uint8_t* A, const uint8_t* sA, f
  *     Y[m,n] = BF16( gA*gW * sum_g sW[n,g] * sum_{k in g} a[m,k]*w[n,k] )
  * with a[m,k] the E4M3 value of byte A_fp8[m][k] (row-major [M][K], one byte per
  * element, any finite E4M3 byte; gA is its FP32 per-tensor scale) and W, sW, gW
- * as for gemm_nvfp4_w4a4 (the activations carry no group scales).  The weight
- * codes are converted by the exact E2M1 -> E4M3 identity and each 16-group's
- * FP8 partial sum is scaled in FP32 by sW*2^6 and accumulated in FP32.
+ * as for gemm_nvfp4_w4a4 (the activations carry no group scales).  Each weight
+ * times its group scale is written exactly as three E5M2 planes (the scale's
+ * signed binary digits times the E2M1 value); three E4M3 x E5M2 FP8 MMAs per
+ * K step accumulate every product exactly into one FP32 accumulator, as the
+ * declared W4A4 product would.
  * M, N >= 0 (0 returns OK and does nothing); K >= 256, K % 256 == 0; every
  * pointer a 16-byte aligned device pointer.  Needs exec_of(device, NVFP4, FP8)
  * == FP8_EXACT (sm_100), else NVFP4_ERR_NOPATH. */
