@@ -493,8 +493,10 @@ def run_ours(args):
     # kernels without the host launch gaps between them, and gives `value`.  The eager
     # loop below still times the product (and the MoE stages) between events.
     graph, launch = None, "eager"
-    # (the grouped step measured no faster replayed than launched eagerly: eager there)
-    if path in ("w4a4", "moe") and not args.no_graph:
+    # (the two-kernel steps launch the product with programmatic dependent launch,
+    # which overlaps its set-up with the scale packing; replayed from a graph they
+    # measured slower than launched eagerly, so only the MoE layer replays a graph)
+    if path in ("moe",) and not args.no_graph:
         try:
             gstream = torch.cuda.Stream(dev)
             gstream.wait_stream(stream)
@@ -534,19 +536,25 @@ def run_ours(args):
                 step()
             ends[i].record(stream)
         torch.cuda.synchronize(dev)
-        if graph is not None:
+        if graph is not None or mids is not None:
+            # `value`: whole steps with nothing between their kernels (an event recorded
+            # between the scale packing and the product would stop the product's launch
+            # from overlapping the packing), or the graph replay
             for i in range(args.steps):
                 flush.zero_()
                 gstarts[i].record(stream)
-                graph.replay()
+                if graph is not None:
+                    graph.replay()
+                else:
+                    step()
                 gends[i].record(stream)
             torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     nv.nvfp4_check_device_error(stream)
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
-    eager_ms = sum(per_step) / len(per_step)
-    if graph is not None:
+    eager_ms = sum(per_step) / len(per_step)   # with the stage events (MoE, W4A4, grouped)
+    if graph is not None or mids is not None:
         per_step = [s.elapsed_time(e) for s, e in zip(gstarts, gends)]
     t_ms = sum(per_step) / len(per_step)
     if world > 1:

@@ -185,6 +185,9 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // the set-up above overlaps the kernel before this one (scale packing or the
+    // schedule, when launched programmatically); their output is read only from here
+    grid_dependency_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)

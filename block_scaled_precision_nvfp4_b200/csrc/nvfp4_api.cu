@@ -583,13 +583,17 @@ nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, 
     cfg.blockDim = dim3(wp::NUM_THREADS);
     cfg.dynamicSmemBytes = wp::SMEM_BYTES;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // may start while the stream's previous kernel (the scale packing) finishes; the
+    // kernel waits for it before reading anything it wrote
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, wp::w4a4_pair_kernel, tmA, tmB, tmSA, tmSB, tmY,
                                        tma_out, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K,
                                        gA * gW);
@@ -995,13 +999,17 @@ nvfp4_status gemm_nvfp4_w4a4_grouped_packed(const uint8_t* A, const uint8_t* sA_
     cfg.blockDim = dim3(gp::NUM_THREADS);
     cfg.dynamicSmemBytes = gp::SMEM_BYTES;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // may start while the stream's previous kernel (the scale packing) finishes; the
+    // kernel waits for it before reading anything it wrote
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, gp::grouped_pair_kernel, tmA, tmA64, tmW, tmSA, tmSW2,
                                        tmSW1, tmY, tma_out, prm, (const gp::Params*)nullptr,
                                        reinterpret_cast<__nv_bfloat16*>(Y));
@@ -1113,13 +1121,17 @@ nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched(const uint8_t* A, const uint8_
     cfg.blockDim = dim3(gp::NUM_THREADS);
     cfg.dynamicSmemBytes = gp::SMEM_BYTES;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // may start while the stream's previous kernel (the scale packing) finishes; the
+    // kernel waits for it before reading anything it wrote
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, gp::grouped_pair_kernel, tmA, tmA64, tmW, tmSA, tmSW2,
                                        tmSW1, tmY, tma_out, none,
                                        (const gp::Params*)sched_params(const_cast<void*>(sched)),

@@ -9,6 +9,7 @@
 // one tcgen05.cp 32x128b.warpx4 puts a K = 64 step's scales for 128 rows into
 // TMEM.  The rearrangement is pure data movement (HBM-bound).
 #pragma once
+#include "ptx.cuh"
 #include <cstdint>
 
 namespace nvfp4 {
@@ -52,6 +53,7 @@ __device__ __forceinline__ void pack_block(const uint8_t* __restrict__ src, int 
 __global__ void __launch_bounds__(ROWS)
 pack_scales_kernel(const uint8_t* __restrict__ s, uint8_t* __restrict__ out, int rows,
                    int groups, int ksteps) {
+    grid_dependents_launch();  // the product that follows may set itself up meanwhile
     const int rb = blockIdx.x;
     pack_block(s + (long long)rb * ROWS * groups, min(ROWS, rows - rb * ROWS),
                out + (long long)rb * ksteps * 512, groups, ksteps, blockIdx.y);
@@ -74,6 +76,7 @@ __global__ void __launch_bounds__(ROWS)
 pack_scales_grouped_kernel(const uint8_t* __restrict__ s, uint8_t* __restrict__ out,
                            const __grid_constant__ GroupedPack gp_param,
                            const GroupedPack* __restrict__ gp_dev, int groups, int ksteps) {
+    grid_dependents_launch();  // the product that follows may set itself up meanwhile
     const GroupedPack& gp = gp_dev ? *gp_dev : gp_param;
     const int b = blockIdx.x;
     if (b >= gp.block_start[gp.groups_n]) return;

@@ -188,6 +188,9 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
     cluster_sync();  // both CTAs' barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // the set-up above overlaps the kernel before this one (the activations' scale
+    // packing, when launched programmatically); its output is read only from here
+    grid_dependency_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
