@@ -27,7 +27,8 @@ __all__ = [
     "nvfp4_exec_name", "nvfp4_set_fp4_kernel_disabled", "nvfp4_version",
     "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_nvfp4_w4a8", "gemm_w4a16",
     "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
-    "gemm_nvfp4_w4a4_packed", "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
+    "gemm_nvfp4_w4a4_packed", "nvfp4_w4a4_packed_workspace_bytes", "w4a4_packed_workspace",
+    "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
     "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "nvfp4_fp4_fallback",
     "nvfp4_node_exec", "moe_route", "moe_permute_rows", "moe_combine", "GroupedSchedule",
     "C_FUNCTIONS",
@@ -92,6 +93,8 @@ C_FUNCTIONS = {
     "nvfp4_scale_layout_bytes": (_Z, [_I, _I]),
     "nvfp4_pack_scales": (_I, [_P, _I, _I, _P, _P]),
     "gemm_nvfp4_w4a4_packed": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
+    "nvfp4_w4a4_packed_workspace_bytes": (_Z, [_I, _I, _I, _I]),
+    "gemm_nvfp4_w4a4_packed_ws": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _I, _P, _Z, _P]),
     "gemm_w4a16": (_I, [_P, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_nvfp4_w4a4_grouped": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
     "nvfp4_grouped_scale_layout_bytes": (_Z, [_P, _I, _I]),
@@ -314,8 +317,26 @@ def nvfp4_quantize_bf16(x, plain=True, packed=True, workspace=None, stream=None,
     return codes, scales, sp, g[:1]
 
 
-def gemm_nvfp4_w4a4_packed(A, sA_packed, gA, W, sW_packed, gW, out=None, stream=None):
-    """gemm_nvfp4_w4a4 with scales packed by nvfp4_pack_scales (pairs of SMs, K % 256 == 0)."""
+def nvfp4_w4a4_packed_workspace_bytes(M, N, K, max_pairs=0):
+    """Device bytes the balanced (stream-K) pair product needs on the current device; 0: none."""
+    return int(load_library().nvfp4_w4a4_packed_workspace_bytes(int(M), int(N), int(K),
+                                                                int(max_pairs)))
+
+
+def w4a4_packed_workspace(M, N, K, max_pairs=0, device=None):
+    """A zeroed workspace for gemm_nvfp4_w4a4_packed(..., workspace=...), or None when
+    the shape needs none.  It stays valid across calls of this shape (or any shape
+    needing no more bytes); calls that overlap on the GPU need one each."""
+    torch = _torch()
+    n = nvfp4_w4a4_packed_workspace_bytes(M, N, K, max_pairs)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda") if n else None
+
+
+def gemm_nvfp4_w4a4_packed(A, sA_packed, gA, W, sW_packed, gW, out=None, stream=None,
+                           workspace=None, max_pairs=0):
+    """gemm_nvfp4_w4a4 with scales packed by nvfp4_pack_scales (pairs of SMs, K % 256 == 0).
+    With a workspace (w4a4_packed_workspace), the last waves of tiles are balanced over
+    the pairs (stream-K); max_pairs > 0 caps the number of SM pairs."""
     torch = _torch()
     M, half_k = A.shape
     N = W.shape[0]
@@ -330,9 +351,19 @@ def gemm_nvfp4_w4a4_packed(A, sA_packed, gA, W, sW_packed, gW, out=None, stream=
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
-    _err(load_library().gemm_nvfp4_w4a4_packed(pa, sA_packed.data_ptr(), float(gA), pw,
-                                               sW_packed.data_ptr(), float(gW), py, M, N, K,
-                                               _stream_ptr(stream)))
+    if workspace is None and not max_pairs:
+        _err(load_library().gemm_nvfp4_w4a4_packed(pa, sA_packed.data_ptr(), float(gA), pw,
+                                                   sW_packed.data_ptr(), float(gW), py, M, N, K,
+                                                   _stream_ptr(stream)))
+        return out
+    if workspace is not None and (not isinstance(workspace, torch.Tensor) or not workspace.is_cuda
+                                  or not workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    pws = workspace.data_ptr() if workspace is not None else None
+    nws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _err(load_library().gemm_nvfp4_w4a4_packed_ws(pa, sA_packed.data_ptr(), float(gA), pw,
+                                                  sW_packed.data_ptr(), float(gW), py, M, N, K,
+                                                  int(max_pairs), pws, nws, _stream_ptr(stream)))
     return out
 
 

@@ -549,10 +549,40 @@ nvfp4_status nvfp4_quantize_bf16_noalloc(const void* X, int rows, int K, uint8_t
                                kNoAllocScratchBytes, stream);
 }
 
-nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, float gA,
-                                    const uint8_t* W, const uint8_t* sW_packed, float gW,
-                                    void* Y, int M, int N, int K, void* stream) {
+namespace {
+// How the pair kernel hands out its tiles: `pairs` clusters; tiles below dp_tiles
+// whole and in turn, the rest as K-block ranges (stream-K) with `slots` cut tiles.
+struct PairPlan {
+    int pairs = 0, tiles = 0, dp_tiles = 0, slots = 0;
+};
+
+PairPlan pair_plan(int M, int N, int K, int num_sms, int max_pairs, bool split) {
     namespace wp = nvfp4::w4a4_pair;
+    PairPlan p;
+    p.tiles = ((M + wp::TILE_M - 1) / wp::TILE_M) * ((N + wp::BN - 1) / wp::BN);
+    p.pairs = p.tiles < num_sms / 2 ? p.tiles : num_sms / 2;
+    if (max_pairs > 0 && p.pairs > max_pairs) p.pairs = max_pairs;
+    p.dp_tiles = p.tiles;
+    if (p.pairs < 1) return p;
+    const int full = p.tiles / p.pairs, rem = p.tiles % p.pairs;
+    // A last wave of whole tiles keeps (pairs - rem) pairs idle for one tile's
+    // time; balanced, that wave costs rem/pairs of a tile instead.  The balancing
+    // itself costs about 0.4 of a tile's time on a B200 (the partial-sum exchange,
+    // one more segment per pair, and no power headroom from idle SMs), so it is
+    // used when the last wave is at most 60 % full.  A cut needs K / 256 >= 2.
+    if (split && full >= 1 && rem != 0 && rem * 5 <= p.pairs * 3 && K / wp::BK >= 2) {
+        p.dp_tiles = (full - 1) * p.pairs;  // leaves rem + pairs tiles: every range >= 1 tile
+        p.slots = p.pairs - 1;
+    }
+    return p;
+}
+
+nvfp4_status launch_w4a4_pair(const uint8_t* A, const uint8_t* sA_packed, float gA,
+                              const uint8_t* W, const uint8_t* sW_packed, float gW, void* Y,
+                              int M, int N, int K, int max_pairs, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    namespace wp = nvfp4::w4a4_pair;
+    if (max_pairs < 0) return fail(NVFP4_ERR_INVALID_ARG, "max_pairs must be >= 0 (got %d)", max_pairs);
     nvfp4_status st = check_w4a4_args(A, sA_packed, W, sW_packed, Y, M, N, K);
     if (st != NVFP4_OK) return st;
     if (K % wp::BK != 0)
@@ -576,10 +606,20 @@ nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, 
     if ((st = make_map_out(&tmY, Y, (uint64_t)M, (uint64_t)N, tma_out)) != NVFP4_OK) return st;
     if ((st = set_smem(wp::w4a4_pair_kernel, wp::SMEM_BYTES, info, "w4a4_pair_kernel")) != NVFP4_OK)
         return st;
-    const int tiles = ((M + wp::TILE_M - 1) / wp::TILE_M) * ((N + wp::BN - 1) / wp::BN);
-    const int pairs = tiles < info.num_sms / 2 ? tiles : info.num_sms / 2;
+    const PairPlan plan = pair_plan(M, N, K, info.num_sms, max_pairs, workspace != nullptr);
+    float* partials = nullptr;
+    unsigned* tickets = nullptr;
+    if (plan.slots > 0) {
+        const size_t need = wp::split_workspace_bytes(plan.slots);
+        if (workspace_bytes < need)
+            return fail(NVFP4_ERR_INVALID_ARG, "the workspace holds %zu bytes; this shape needs %zu",
+                        workspace_bytes, need);
+        if (!aligned16(workspace)) return fail(NVFP4_ERR_MISALIGNED, "the workspace must be 16-byte aligned");
+        tickets = static_cast<unsigned*>(workspace);
+        partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + wp::ticket_bytes(plan.slots));
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs);
+    cfg.gridDim = dim3(2 * plan.pairs);
     cfg.blockDim = dim3(wp::NUM_THREADS);
     cfg.dynamicSmemBytes = wp::SMEM_BYTES;
     cfg.stream = static_cast<cudaStream_t>(stream);
@@ -596,9 +636,32 @@ nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, 
     cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, wp::w4a4_pair_kernel, tmA, tmB, tmSA, tmSB, tmY,
                                        tma_out, reinterpret_cast<__nv_bfloat16*>(Y), M, N, K,
-                                       gA * gW);
+                                       gA * gW, plan.dp_tiles, partials, tickets);
     if (e != cudaSuccess) return cuda_fail(e, "launching w4a4_pair_kernel");
     return ok();
+}
+}  // namespace
+
+nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, float gA,
+                                    const uint8_t* W, const uint8_t* sW_packed, float gW,
+                                    void* Y, int M, int N, int K, void* stream) {
+    return launch_w4a4_pair(A, sA_packed, gA, W, sW_packed, gW, Y, M, N, K, 0, nullptr, 0, stream);
+}
+
+size_t nvfp4_w4a4_packed_workspace_bytes(int M, int N, int K, int max_pairs) {
+    int dev;
+    DevInfo info;
+    if (M <= 0 || N <= 0 || K <= 0 || max_pairs < 0 || !current_device(dev, info)) return 0;
+    const PairPlan plan = pair_plan(M, N, K, info.num_sms, max_pairs, true);
+    return plan.slots > 0 ? nvfp4::w4a4_pair::split_workspace_bytes(plan.slots) : 0;
+}
+
+nvfp4_status gemm_nvfp4_w4a4_packed_ws(const uint8_t* A, const uint8_t* sA_packed, float gA,
+                                       const uint8_t* W, const uint8_t* sW_packed, float gW,
+                                       void* Y, int M, int N, int K, int max_pairs,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+    return launch_w4a4_pair(A, sA_packed, gA, W, sW_packed, gW, Y, M, N, K, max_pairs, workspace,
+                            workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------------------- via FP8

@@ -22,6 +22,22 @@
 // scales packed ahead there is no shared-memory rewrite or cross-CTA hand-off
 // on the critical path.  All waits are bounded; both CTAs meet at a cluster
 // barrier before the pair's TMEM is freed.
+//
+// Load balance (stream-K over the last waves): when the tiles do not divide
+// evenly among the pairs, the last wave of whole tiles would leave most pairs
+// idle.  With a workspace, the tiles are then handed out in two parts:
+//   * the K-blocks of the last one-and-a-half waves of tiles, laid end to end,
+//     are cut into one contiguous range per pair, so every pair multiplies the
+//     same number of K-blocks (give or take one).  A range is at least one tile
+//     long, so a tile cut by a range boundary has exactly two contributors;
+//   * the other tiles go whole to the pairs in turn, after each pair's range
+//     (so the partial-sum exchange below is hidden behind them).
+// Each epilogue warp of a cut tile takes a ticket in the workspace: the first of
+// the two contributors to arrive writes its FP32 partial sums there, and the
+// second adds them to its own and writes the BF16 output.  Nobody waits for
+// anybody, and the sum of two FP32 terms is the same in either order, so the
+// output does not depend on which contributor comes first.  The second one
+// resets the ticket, so the workspace is ready for the next launch.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -77,6 +93,132 @@ __host__ __device__ constexpr uint32_t sfa_col(int s) { return BN + s * (SFA_COL
 __host__ __device__ constexpr uint32_t sfb_col(int s) { return sfa_col(s) + SFA_COLS; }
 
 constexpr int SLAB_COLS = 64;  // columns of one output store box (128 bytes)
+
+// ---- stream-K workspace: per cut tile ("slot"), a ticket for each epilogue warp of
+// each CTA, and the two contributors' FP32 partials of that warp's 32 x 128 block,
+// stored as [32 column quads][32 lanes] float4 (a warp's store of one quad is 512
+// contiguous bytes).
+constexpr int PART_FLOATS = 32 * (BN / 2);
+constexpr int TICKETS_PER_SLOT = 2 * NUM_EPI_WARPS;
+__host__ __device__ constexpr size_t part_offset(int slot, int side, int rank, int w) {
+    return ((((size_t)slot * 2 + side) * 2 + rank) * NUM_EPI_WARPS + w) * PART_FLOATS;
+}
+// bytes of tickets (rounded up to 256) and partials for `slots` cut tiles
+__host__ __device__ constexpr size_t ticket_bytes(int slots) {
+    return ((size_t)slots * TICKETS_PER_SLOT * 4 + 255) & ~(size_t)255;
+}
+__host__ __device__ constexpr size_t split_workspace_bytes(int slots) {
+    return ticket_bytes(slots) + part_offset(slots, 0, 0, 0) * sizeof(float);
+}
+
+// One unit of a pair's work: K-blocks [kb0, kb1) of one output tile.
+struct Segment {
+    int tile, kb0, kb1;
+    int slot;  // -1: the tile is this pair's alone; else its partial-sum slot
+    int side;  // 0: the tile's first K-blocks, 1: its last ones
+};
+
+// The j-th segment of pair `cid` of `P`: first this pair's range of the K-blocks
+// of the tiles from dp_tiles on (range c is [c*S/P, (c+1)*S/P) of the S K-blocks
+// laid end to end), then the tiles below dp_tiles whole, in turn (cid, cid + P,
+// ...).  The cut tiles come first, the shorter cut before the longer and both
+// before the range's whole tiles: the epilogue of a cut segment exchanges partial
+// sums, and what follows it on the MMA should be long enough to hide that (with a
+// single accumulator, a late epilogue holds up the MMAs of the segment after
+// next).  The cut at the start of range c (c >= 1) is slot c - 1.  False past the
+// pair's last segment.
+__device__ __forceinline__ bool segment_of(int j, int cid, int P, int tiles, int dp_tiles,
+                                           int num_kb, Segment& sg) {
+    const long long S = (long long)(tiles - dp_tiles) * num_kb;
+    const long long b = S * cid / P, e = S * (cid + 1) / P;
+    const int n_sk = S > 0 ? (int)((e - 1) / num_kb - b / num_kb + 1) : 0;
+    sg.slot = -1;
+    sg.side = 0;
+    if (j >= n_sk) {
+        const int jd = j - n_sk;
+        const int n_dp = cid < dp_tiles ? (dp_tiles - cid + P - 1) / P : 0;
+        if (jd >= n_dp) return false;
+        sg.tile = cid + jd * P;
+        sg.kb0 = 0;
+        sg.kb1 = num_kb;
+        return true;
+    }
+    // the range's segments in K order are 0 .. n_sk-1; 0 is cut when b is inside a
+    // tile, n_sk-1 when e is (a range of at least one tile has two distinct ends)
+    const int head = (int)(b % num_kb), tail = (int)(e % num_kb);
+    int k = j;
+    if (head && tail) {
+        const bool head_shorter = num_kb - head <= tail;
+        k = j == 0 ? (head_shorter ? 0 : n_sk - 1) : j == 1 ? (head_shorter ? n_sk - 1 : 0) : j - 1;
+    } else if (tail) {
+        k = j == 0 ? n_sk - 1 : j - 1;
+    }
+    const long long t = b / num_kb + k;  // among the tiles from dp_tiles on
+    const long long t0 = t * num_kb;     // its first K-block, end to end
+    sg.tile = dp_tiles + (int)t;
+    sg.kb0 = b > t0 ? (int)(b - t0) : 0;
+    sg.kb1 = e - t0 < num_kb ? (int)(e - t0) : num_kb;
+    if (sg.kb0 > 0) {
+        sg.slot = cid - 1;
+        sg.side = 1;
+    } else if (sg.kb1 < num_kb) {
+        sg.slot = cid;
+        sg.side = 0;
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// A cut tile's epilogue warp, holding its own FP32 partial sums in r (column
+// 32c + k in r[c][k]).  Returns false when it is the first contributor to arrive:
+// its partial is then left in the workspace.  Returns true when it is the second:
+// r then holds the sum of both partials, and the ticket is back at zero.
+__device__ __forceinline__ bool combine_partial(float* __restrict__ ws, unsigned* __restrict__ tickets,
+                                                const Segment& sg, int rank, int w,
+                                                uint32_t (&r)[4][32]) {
+    const int lane = threadIdx.x & 31;
+    unsigned* tk = tickets + (sg.slot * 2 + rank) * NUM_EPI_WARPS + w;
+    unsigned seen = 0;
+    if (lane == 0) seen = ld_acquire_gpu(tk);
+    seen = __shfl_sync(0xffffffffu, seen, 0);
+    if (seen == 0) {
+        float4* mine = reinterpret_cast<float4*>(ws + part_offset(sg.slot, sg.side, rank, w)) + lane;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            __stcg(mine + i * 32, make_float4(__uint_as_float(r[i >> 3][(i & 7) * 4]),
+                                              __uint_as_float(r[i >> 3][(i & 7) * 4 + 1]),
+                                              __uint_as_float(r[i >> 3][(i & 7) * 4 + 2]),
+                                              __uint_as_float(r[i >> 3][(i & 7) * 4 + 3])));
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) seen = atomicAdd(tk, 1u);
+        seen = __shfl_sync(0xffffffffu, seen, 0);
+        if (seen == 0) return false;
+    }
+    __threadfence();
+    const float4* other =
+        reinterpret_cast<const float4*>(ws + part_offset(sg.slot, sg.side ^ 1, rank, w)) + lane;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 o = __ldcg(other + (c * 8 + q) * 32);
+            r[c][4 * q] = __float_as_uint(__uint_as_float(r[c][4 * q]) + o.x);
+            r[c][4 * q + 1] = __float_as_uint(__uint_as_float(r[c][4 * q + 1]) + o.y);
+            r[c][4 * q + 2] = __float_as_uint(__uint_as_float(r[c][4 * q + 2]) + o.z);
+            r[c][4 * q + 3] = __float_as_uint(__uint_as_float(r[c][4 * q + 3]) + o.w);
+        }
+        reg_fence(r[c]);
+    }
+    __syncwarp();
+    if (lane == 0) atomicExch(tk, 0u);
+    return true;
+}
 
 // One epilogue warp's 32 rows (lane = row) x 128 columns, held as packed BF16
 // pairs, stored through the warp's 4 KB staging buffer as two 32 x 64 boxes.
@@ -152,7 +294,10 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
                  const __grid_constant__ CUtensorMap tmSB,  // packed sW: same view, box (128, 16, 2)
                  const __grid_constant__ CUtensorMap tmY,   // Y bf16 [M][N], box 64 x 32, 128B swizzle
                  int tma_out,                               // tmY is valid (N % 8 == 0)
-                 __nv_bfloat16* __restrict__ Y, int M, int N, int K, float alpha) {
+                 __nv_bfloat16* __restrict__ Y, int M, int N, int K, float alpha,
+                 int dp_tiles,                     // tiles handed out whole (all of them: no split)
+                 float* __restrict__ ws,           // partial sums of cut tiles (split only)
+                 unsigned* __restrict__ tickets) { // one per epilogue warp of a cut tile, zero between launches
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~uintptr_t(1023));
@@ -196,11 +341,12 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
         // ------------------------------------------------------------ producer (both CTAs)
         int it = 0;
         bool ok = true;
-        for (int tile = cid; tile < tiles && ok; tile += nclusters) {
+        Segment sg;
+        for (int j = 0; ok && segment_of(j, cid, nclusters, tiles, dp_tiles, num_kb, sg); ++j) {
             int mb, nb;
-            tile_coords(tile, num_m, num_n, mb, nb);
+            tile_coords(sg.tile, num_m, num_n, mb, nb);
             const int arb = mb * 2 + (int)rank;  // this CTA's 128-row block of A
-            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+            for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
                 const int s = it % STAGES;
                 if (!warp_wait(&sm.empty[s], ((it / STAGES) & 1) ^ 1, abort, ROLE_PRODUCER, 32)) {
                     ok = false;
@@ -233,10 +379,12 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
             const uint32_t idesc = idesc_mxf4nvf4(TILE_M, BN);
             int it = 0, tc = 0;
             bool ok = true;
-            for (int tile = cid; tile < tiles && ok; tile += nclusters, ++tc) {
+            Segment sg;
+            for (int j = 0; ok && segment_of(j, cid, nclusters, tiles, dp_tiles, num_kb, sg);
+                 ++j, ++tc) {
                 if (!warp_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
                 tc_fence_after();
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
                     const int s = it % STAGES;
                     if (!warp_wait(&sm.full[s], (it / STAGES) & 1, abort, ROLE_MMA)) { ok = false; break; }
                     tc_fence_after();
@@ -258,7 +406,8 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
                             mma_mxf4nvf4_pair(tmem, desc_kmajor_sw128(a0 + ks * 32),
                                               desc_kmajor_sw128(b0 + ks * 32), idesc,
                                               tmem + sfa_col(s) + ks * 4,
-                                              tmem + sfb_col(s) + ks * NRB * 4, (kb | ks) != 0);
+                                              tmem + sfb_col(s) + ks * NRB * 4,
+                                              kb != sg.kb0 || ks != 0);
                         mma_commit_pair(&sm.empty[s], 0x3);
                     }
                     __syncwarp();
@@ -286,28 +435,35 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
         static_assert(COLS == 128, "one epilogue warp stores 128 columns");
         uint8_t* stage = sm.out[warp - FIRST_EPI_WARP];
         int tc = 0;
-        for (int tile = cid; tile < tiles; tile += nclusters, ++tc) {
+        Segment sg;
+        for (int j = 0; segment_of(j, cid, nclusters, tiles, dp_tiles, num_kb, sg); ++j, ++tc) {
             int mb, nb;
-            tile_coords(tile, num_m, num_n, mb, nb);
+            tile_coords(sg.tile, num_m, num_n, mb, nb);
             if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI, 256)) break;
             tc_fence_after();
-            uint32_t packed[COLS / 2];
+            // the whole accumulator block behind one wait, then TMEM goes back to the MMA
+            uint32_t r[CHUNKS][32];
 #pragma unroll
-            for (int c = 0; c < CHUNKS; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + half * COLS + c * 32, r);
-                tmem_ld_wait();
-                reg_fence(r);
+            for (int c = 0; c < CHUNKS; ++c)
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + half * COLS + c * 32, r[c]);
+            tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
-                                                             __uint_as_float(r[2 * j + 1]) * alpha);
-                    packed[c * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
-                }
-            }
+            for (int c = 0; c < CHUNKS; ++c) reg_fence(r[c]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(&sm.acc_empty, 0);
+            if (sg.slot >= 0 &&
+                !combine_partial(ws, tickets, sg, (int)rank, warp - FIRST_EPI_WARP, r))
+                continue;  // the other contributor of this cut tile finishes it
+            uint32_t packed[COLS / 2];
+#pragma unroll
+            for (int c = 0; c < CHUNKS; ++c)
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[c][2 * k]) * alpha,
+                                                             __uint_as_float(r[c][2 * k + 1]) * alpha);
+                    packed[c * 16 + k] = *reinterpret_cast<uint32_t*>(&h);
+                }
 
             const int row0 = mb * TILE_M + (int)rank * BM + 32 * q;
             const int col0 = nb * BN + half * COLS;

@@ -243,6 +243,45 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* s
                                               const uint8_t* W, const uint8_t* sW_packed, float gW,
                                               void* Y_bf16, int M, int N, int K, void* stream);
 
+/* Device bytes of the workspace that gemm_nvfp4_w4a4_packed_ws needs for this
+ * shape on the current device with at most `max_pairs` SM pairs (0: one pair per
+ * two SMs).  0 when the tiles divide evenly among the pairs, or when no split
+ * pays: fewer tiles than pairs, a last wave of whole tiles that would be more
+ * than 60 % full, or a single K-block. The call then needs none.
+ * The need grows with the number of pairs, not with the tensors: 512 KB per pair,
+ * about 38 MB on a 148-SM part.  0 also when the device cannot be queried. */
+NVFP4_API size_t nvfp4_w4a4_packed_workspace_bytes(int M, int N, int K, int max_pairs);
+
+/* gemm_nvfp4_w4a4_packed with the last waves of tiles balanced over the pairs
+ * (stream-K).  This is a design of this library, not of the pages; the product
+ * is the page-1 module doc's NVFP4 row, as for gemm_nvfp4_w4a4_packed.
+ *   - Whole 256 x 256 tiles go to the pairs in turn until about one and a half
+ *     waves of tiles are left. The K-blocks of those are laid end to end and
+ *     cut into one contiguous range per pair, so that no pair idles through a
+ *     part-empty last wave.
+ *   - A tile cut between two pairs is summed in FP32 from the two partial
+ *     products (the first K-blocks and the rest). That changes only where the
+ *     FP32 accumulation is split. Each output element is still the FP32 sum
+ *     over all of K, times gA*gW, rounded once to BF16. The sum of the two
+ *     FP32 terms does not depend on which pair finishes first, so the output
+ *     is the same on every run.
+ *   - max_pairs: 0 = one pair per two SMs; otherwise at most that many pairs
+ *     (for instance to leave SMs to concurrent work).
+ *   - workspace: device memory, 16-byte aligned, of workspace_bytes >=
+ *     nvfp4_w4a4_packed_workspace_bytes(M, N, K, max_pairs) (NULL when that is
+ *     0; a smaller buffer is NVFP4_ERR_INVALID_ARG). The caller owns it. It
+ *     must be all zero before its first use. Each call leaves it ready for the
+ *     next (its tickets back at zero). Zero it again after a call that
+ *     reported NVFP4_ERR_DEVICE_TIMEOUT. Calls whose work overlaps on the GPU
+ *     need one workspace each.
+ *   - Everything else (operands, errors) as gemm_nvfp4_w4a4_packed. */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a4_packed_ws(const uint8_t* A, const uint8_t* sA_packed,
+                                                 float gA, const uint8_t* W,
+                                                 const uint8_t* sW_packed, float gW, void* Y_bf16,
+                                                 int M, int N, int K, int max_pairs,
+                                                 void* workspace, size_t workspace_bytes,
+                                                 void* stream);
+
 /* The same product through the exact E2M1->E4M3 conversion on the FP8 MMA
  * (module doc, bullet 2): each packed code byte is split into its two nibbles,
  * each placed in the high nibble of a byte and converted by
