@@ -427,7 +427,6 @@ def run_ours(args):
                                dtype=torch.uint8, device=dev)
         gc_b = torch.empty_like(codes_b)
         gs_b = torch.empty_like(scales_b)
-        Yg_b = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ones = torch.ones((M, 1), dtype=torch.float32, device=dev)
 
         sa_b = torch.empty(nv.load_library().nvfp4_grouped_scale_layout_bytes_bound(M, E, K),
@@ -453,10 +452,10 @@ def run_ours(args):
             sched = nv.GroupedSchedule(off, E, M, N, K, gws, gA=g_b[:1], stream=s)
             sched.pack(gs_b, out=sa_b, stream=s)
             mark(4)
-            sched.gemm(gc_b, sa_b, Wc_d, sw_packed, out=Yg_b, stream=s)
+            # top-1: the combine (weight, then each row to its token) is fused into the
+            # grouped product's epilogue, so the expert-order rows never reach memory
+            sched.gemm_combine(gc_b, sa_b, Wc_d, sw_packed, src, M, weights=ones, out=Y, stream=s)
             mark(5)
-            nv.moe_combine(Yg_b, dest, ones, M, 1, out=Y, stream=s)
-            mark(6)
     elif path == "w4a8":
         def step():
             nv.gemm_nvfp4_w4a8(dv[0], wl_.gA, dv[1], dv[2], wl_.W.g, out=Y, stream=stream)
@@ -484,7 +483,7 @@ def run_ours(args):
         def plain_step():
             nv.gemm_nvfp4_w4a4(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
     launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2, "grouped": 2, "quantize": 2,
-                         "moe": 11}.get(path, 1)
+                         "moe": 8}.get(path, 1)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -524,7 +523,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     mids = ([torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
             if path in ("w4a4", "grouped") else None)
-    stage_ev = ([[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    stage_ev = ([[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
                 if path == "moe" else None)
     gstarts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     gends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -664,13 +663,12 @@ def run_ours(args):
                  "plain_scale_entry_ms": statistics.median(plain),
                  "plain_scale_entry_tflops": flops / (statistics.median(plain) * 1e-3) / 1e12}
     if stage_ev is not None:
-        names = ["quantize", "route", "permute", "schedule_and_pack", "grouped_gemm", "combine"]
+        names = ["quantize", "route", "permute", "schedule_and_pack", "grouped_gemm_and_combine"]
         med = {n: statistics.median(ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev) * 1e3
                for j, n in enumerate(names)}
-        kern_s = med["grouped_gemm"] * 1e-6
+        kern_s = med["grouped_gemm_and_combine"] * 1e-6
         extra = {"stage_us": med,
-                 "permute_gbs": 2 * M * (K // 2 + K // 16) / (med["permute"] * 1e-6) / 1e9,
-                 "combine_gbs": 2 * M * N * 2 / (med["combine"] * 1e-6) / 1e9}
+                 "permute_gbs": 2 * M * (K // 2 + K // 16) / (med["permute"] * 1e-6) / 1e9}
     kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel", "w4a8": "w4a8_kernel",
                    "moe": "grouped_pair_kernel",
                    "w4a16": "w4a16_kernel", "grouped": "grouped_pair_kernel",
@@ -747,7 +745,8 @@ def run_ours(args):
                   if path == "w4a16" else
                   "e4m3 x nvfp4(e2m1, e4m3 group scales) -> f32 accumulate -> bf16"
                   if path == "w4a8" else
-                  "bf16 -> nvfp4 -> grouped nvfp4 x nvfp4 -> f32 -> bf16 -> f32 combine -> bf16"
+                  "bf16 -> nvfp4 -> grouped nvfp4 x nvfp4 -> f32 -> x routing weight -> bf16 "
+                  "(top-1 combine fused)"
                   if path == "moe" else
                   "nvfp4(e2m1 x e2m1, e4m3 group scales) -> f32 accumulate -> bf16"),
         "data": "synthetic",

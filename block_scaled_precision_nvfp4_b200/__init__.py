@@ -110,6 +110,8 @@ C_FUNCTIONS = {
     "nvfp4_grouped_schedule": (_I, [_P, _I, _I, _I, _I, _P, _F, _P, _P, _P]),
     "nvfp4_pack_scales_grouped_sched": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "gemm_nvfp4_w4a4_grouped_packed_sched": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _P]),
+    "gemm_nvfp4_w4a4_grouped_packed_sched_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _P, _P, _P,
+                                                          _I, _I, _I, _P]),
     "nvfp4_quantize_bf16": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "nvfp4_quantize_bf16_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _P]),
 }
@@ -602,4 +604,22 @@ class GroupedSchedule:
         _err(load_library().gemm_nvfp4_w4a4_grouped_packed_sched(
             pa, sA_packed.data_ptr(), pw, sW_packed.data_ptr(), self.buf.data_ptr(), self.E,
             self.M, py, self.N, self.K, _stream_ptr(stream)))
+        return out
+
+    def gemm_combine(self, A, sA_packed, W, sW_packed, src, T, weights=None, out=None,
+                     stream=None):
+        """gemm with the top-1 combine in its epilogue: grouped row r goes to out row
+        src[r], times weights[src[r]] (device float [T]; None: 1).  out [T, N] bf16."""
+        torch = _torch()
+        pa = _dev_tensor(A, torch.uint8, (self.M, self.K // 2), "A")
+        pw = _dev_tensor(W, torch.uint8, (self.E, self.N, self.K // 2), "W")
+        psrc = _dev_tensor(src, torch.int32, (self.M,), "src")
+        pwt = (_dev_tensor(weights.reshape(-1), torch.float32, (int(T),), "weights")
+               if weights is not None else None)
+        if out is None:
+            out = torch.empty((int(T), self.N), dtype=torch.bfloat16, device=A.device)
+        py = _dev_tensor(out, torch.bfloat16, (int(T), self.N), "out")
+        _err(load_library().gemm_nvfp4_w4a4_grouped_packed_sched_combine(
+            pa, sA_packed.data_ptr(), pw, sW_packed.data_ptr(), self.buf.data_ptr(), self.E,
+            self.M, psrc, pwt, py, int(T), self.N, self.K, _stream_ptr(stream)))
         return out

@@ -113,6 +113,61 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
     return tl;
 }
 
+constexpr int BAD_DEST = 0x40000;  // device error bit: a grouped row's Y row outside [0, dest_rows)
+
+// The Y row and output factor of one grouped row, for a fused combine: row `dest`
+// (the grouped row's index on entry) goes to Y row row_dest[dest], scaled by
+// alpha * row_w[that row].  A row outside [0, dest_rows) is recorded in the device
+// error word and left out (dest = -1); rows past the tile (`valid` false) are not read.
+__device__ __forceinline__ void row_target(const int32_t* __restrict__ row_dest,
+                                           const float* __restrict__ row_w, int dest_rows,
+                                           bool valid, float alpha, int& dest, float& f) {
+    if (!valid) {
+        dest = -1;
+        return;
+    }
+    const int d = __ldg(row_dest + dest);
+    if ((unsigned)d >= (unsigned)dest_rows) {
+        atomicOr(&g_device_error, BAD_DEST);
+        dest = -1;
+        return;
+    }
+    dest = d;
+    if (row_w) f = alpha * __ldg(row_w + d);
+}
+
+// store_slab for scattered rows: the warp's 32 rows x 128 columns (packed BF16
+// pairs, lane = row) pass through the warp's staging buffer one 64-column box at a
+// time, and each row leaves as one 128-byte store to Y row `dest` of its lane
+// (rows with dest < 0, rows past `nrows` and columns past N are not written).
+// N must be even.
+__device__ __forceinline__ void scatter_slab(uint8_t* stage, const uint32_t (&packed)[64], int dest,
+                                             int nrows, int col0, int N, __nv_bfloat16* __restrict__ Y) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (lane == 0) bulk_wait_read_all();  // no TMA store still reads the buffer
+        __syncwarp();
+        uint8_t* rowp = stage + lane * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int w = h * 32 + c * 4;
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(packed[w], packed[w + 1], packed[w + 2], packed[w + 3]);
+        }
+        __syncwarp();
+        const int x = col0 + h * 64 + 2 * lane;  // this lane's two columns
+        for (int r = 0; r < nrows; ++r) {
+            const int d = __shfl_sync(0xffffffffu, dest, r);
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(
+                stage + r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + (lane & 3) * 4);
+            if (d >= 0 && x < N)
+                *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(Y) + (size_t)d * N + x) = v;
+        }
+        __syncwarp();  // the box is read before the next one overwrites it
+    }
+}
+
 // One stage's scale copies and MMAs (issued by one thread of the leader):
 // sA of the MMA's M rows (this CTA's 128), sB of its N side in NB 128-row
 // blocks, then four K = 64 block-scaled MMAs.  Unrolled for each NB so the
@@ -149,7 +204,11 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
                     int tma_out,                                // tmY is valid (N % 8 == 0)
                     const __grid_constant__ Params p_param,
                     const Params* __restrict__ p_dev,           // schedule in device memory, or null
-                    __nv_bfloat16* __restrict__ Y) {
+                    __nv_bfloat16* __restrict__ Y,
+                    // with row_dest: grouped row r goes to Y row row_dest[r] (of dest_rows),
+                    // times row_w[row_dest[r]] when row_w is given (a fused top-1 combine)
+                    const int32_t* __restrict__ row_dest, const float* __restrict__ row_w,
+                    int dest_rows) {
     // the tile schedule: kernel parameters planned on the host, or device memory
     // written by grouped_schedule_kernel from device-resident expert offsets
     const Params& p = p_dev ? *p_dev : p_param;
@@ -283,9 +342,14 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
         for (int t = cid; t < tiles; t += nclusters, ++tc) {
             const Tile tl = decode(p, t);
             const float alpha = p.alpha[tl.e];
-            if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI, 256)) break;
-            tc_fence_after();
             if (!tl.swap) {
+                const int rbase = (int)rank * BM + 32 * q;  // the warp's first row within the tile
+                // this lane's row: its Y row and factor (read before the accumulator is ready)
+                int dest = tl.m0 + rbase + lane;
+                float f = alpha;
+                if (row_dest) row_target(row_dest, row_w, dest_rows, rbase + lane < tl.rows, alpha, dest, f);
+                if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI, 256)) break;
+                tc_fence_after();
                 uint32_t packed[COLS / 2];
 #pragma unroll
                 for (int c = 0; c < CHUNKS; ++c) {
@@ -295,24 +359,36 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
                     reg_fence(r);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
-                                                                 __uint_as_float(r[2 * j + 1]) * alpha);
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * f,
+                                                                 __uint_as_float(r[2 * j + 1]) * f);
                         packed[c * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(&sm.acc_empty, 0);
-                const int rbase = (int)rank * BM + 32 * q;  // the warp's first row within the tile
                 const int col0 = tl.n0 + half * COLS;
-                if (rbase < tl.rows)
-                    store_slab(&tmY, tma_out != 0 && rbase + 32 <= tl.rows, stage, packed,
-                               tl.m0 + rbase, min(32, tl.rows - rbase), col0, N, Y);
+                if (rbase < tl.rows) {
+                    if (row_dest)
+                        scatter_slab(stage, packed, dest, min(32, tl.rows - rbase), col0, N, Y);
+                    else
+                        store_slab(&tmY, tma_out != 0 && rbase + 32 <= tl.rows, stage, packed,
+                                   tl.m0 + rbase, min(32, tl.rows - rbase), col0, N, Y);
+                }
             } else {
-                // lanes are this CTA's weight rows, columns are the tile's token slots
+                // lanes are this CTA's weight rows, columns are the tile's token slots; this
+                // lane holds the Y row and factor of token slots lane and 32 + lane
                 const int n = tl.n0 + (int)rank * BNH + 32 * q + lane;
                 const bool nok = n < N;
-                uint16_t* ycol = reinterpret_cast<uint16_t*>(Y) + (size_t)tl.m0 * N + n;
+                const int tok0 = half * 64;
+                int d0 = tl.m0 + tok0 + lane, d1 = d0 + 32;
+                float f0 = alpha, f1 = alpha;
+                if (row_dest) {
+                    row_target(row_dest, row_w, dest_rows, tok0 + lane < tl.rows, alpha, d0, f0);
+                    row_target(row_dest, row_w, dest_rows, tok0 + 32 + lane < tl.rows, alpha, d1, f1);
+                }
+                if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI, 256)) break;
+                tc_fence_after();
                 uint32_t tok2[32];  // BF16 pairs of consecutive tokens
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
@@ -322,20 +398,23 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
                     reg_fence(r);
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
-                                                                 __uint_as_float(r[2 * j + 1]) * alpha);
+                        // token slots 32c + 2j and 32c + 2j + 1; their factors sit in lanes 2j, 2j + 1
+                        const float fa = __shfl_sync(0xffffffffu, c ? f1 : f0, 2 * j);
+                        const float fb = __shfl_sync(0xffffffffu, c ? f1 : f0, 2 * j + 1);
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * fa,
+                                                                 __uint_as_float(r[2 * j + 1]) * fb);
                         tok2[c * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(&sm.acc_empty, 0);
-                const int tok0 = half * 64;
-                if (nok) {
+                uint16_t* y16 = reinterpret_cast<uint16_t*>(Y);
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        if (tok0 + j < tl.rows)
-                            ycol[(size_t)(tok0 + j) * N] = (uint16_t)(tok2[j >> 1] >> (16 * (j & 1)));
+                for (int j = 0; j < 64; ++j) {
+                    const int d = __shfl_sync(0xffffffffu, j < 32 ? d0 : d1, j & 31);
+                    if (nok && tok0 + j < tl.rows && d >= 0)
+                        y16[(size_t)d * N + n] = (uint16_t)(tok2[j >> 1] >> (16 * (j & 1)));
                 }
             }
         }

@@ -363,6 +363,8 @@ nvfp4_status nvfp4_check_device_error(void* stream) {
     if (v & nvfp4::grouped_pair::BAD_OFFSETS)
         return fail(NVFP4_ERR_INVALID_ARG,
                     "device expert offsets were not a non-decreasing run from 0 to M");
+    if (v & nvfp4::grouped_pair::BAD_DEST)
+        return fail(NVFP4_ERR_INVALID_ARG, "a grouped row's output row (src) was outside [0, T)");
     return fail(NVFP4_ERR_INVALID_ARG, "a routed expert id was outside [0, E)");
 }
 
@@ -1075,7 +1077,8 @@ nvfp4_status gemm_nvfp4_w4a4_grouped_packed(const uint8_t* A, const uint8_t* sA_
     cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, gp::grouped_pair_kernel, tmA, tmA64, tmW, tmSA, tmSW2,
                                        tmSW1, tmY, tma_out, prm, (const gp::Params*)nullptr,
-                                       reinterpret_cast<__nv_bfloat16*>(Y));
+                                       reinterpret_cast<__nv_bfloat16*>(Y), (const int32_t*)nullptr,
+                                       (const float*)nullptr, 0);
     if (e != cudaSuccess) return cuda_fail(e, "launching grouped_pair_kernel");
     return ok();
 }
@@ -1141,10 +1144,13 @@ nvfp4_status nvfp4_pack_scales_grouped_sched(const uint8_t* s_plain, int M, int 
     return e == cudaSuccess ? ok() : cuda_fail(e, "launching pack_scales_grouped_kernel");
 }
 
-nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched(const uint8_t* A, const uint8_t* sA_packed,
-                                                  const uint8_t* W, const uint8_t* sW_packed,
-                                                  const void* sched, int E, int M, void* Y, int N,
-                                                  int K, void* stream) {
+namespace {
+// The device-scheduled grouped product; with row_dest, grouped row r is written to
+// Y row row_dest[r] (of dest_rows), times row_w[that row] if row_w is given.
+nvfp4_status launch_grouped_sched(const uint8_t* A, const uint8_t* sA_packed, const uint8_t* W,
+                                  const uint8_t* sW_packed, const void* sched, int E, int M, void* Y,
+                                  int N, int K, const int32_t* row_dest, const float* row_w,
+                                  int dest_rows, void* stream) {
     namespace gp = nvfp4::grouped_pair;
     if (E < 1 || E > gp::MAX_EXPERTS)
         return fail(NVFP4_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", gp::MAX_EXPERTS, E);
@@ -1173,7 +1179,9 @@ nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched(const uint8_t* A, const uint8_
     if ((st = make_map_packed_sf(&tmSW1, sW_packed, wblocks, ks, 1)) != NVFP4_OK) return st;
     CUtensorMap tmY;
     int tma_out = 0;
-    if ((st = make_map_out(&tmY, Y, (uint64_t)M, (uint64_t)N, tma_out)) != NVFP4_OK) return st;
+    if ((st = make_map_out(&tmY, Y, (uint64_t)(row_dest ? dest_rows : M), (uint64_t)N, tma_out)) !=
+        NVFP4_OK)
+        return st;
     if ((st = set_smem(gp::grouped_pair_kernel, gp::SMEM_BYTES, info, "grouped_pair_kernel")) != NVFP4_OK)
         return st;
     gp::Params none;
@@ -1198,9 +1206,32 @@ nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched(const uint8_t* A, const uint8_
     cudaError_t e = cudaLaunchKernelEx(&cfg, gp::grouped_pair_kernel, tmA, tmA64, tmW, tmSA, tmSW2,
                                        tmSW1, tmY, tma_out, none,
                                        (const gp::Params*)sched_params(const_cast<void*>(sched)),
-                                       reinterpret_cast<__nv_bfloat16*>(Y));
+                                       reinterpret_cast<__nv_bfloat16*>(Y), row_dest, row_w,
+                                       dest_rows);
     if (e != cudaSuccess) return cuda_fail(e, "launching grouped_pair_kernel");
     return ok();
+}
+}  // namespace
+
+nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched(const uint8_t* A, const uint8_t* sA_packed,
+                                                  const uint8_t* W, const uint8_t* sW_packed,
+                                                  const void* sched, int E, int M, void* Y, int N,
+                                                  int K, void* stream) {
+    return launch_grouped_sched(A, sA_packed, W, sW_packed, sched, E, M, Y, N, K, nullptr, nullptr,
+                                0, stream);
+}
+
+nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched_combine(const uint8_t* A,
+                                                          const uint8_t* sA_packed, const uint8_t* W,
+                                                          const uint8_t* sW_packed, const void* sched,
+                                                          int E, int M, const int32_t* src,
+                                                          const float* weights, void* Y, int T,
+                                                          int N, int K, void* stream) {
+    if (M > 0 && !src) return fail(NVFP4_ERR_INVALID_ARG, "null src");
+    if (T < 0 || M > T) return fail(NVFP4_ERR_INVALID_ARG, "top-1 needs M <= T (got M %d, T %d)", M, T);
+    if (N % 2 != 0) return fail(NVFP4_ERR_INVALID_ARG, "the fused combine needs an even N (got %d)", N);
+    return launch_grouped_sched(A, sA_packed, W, sW_packed, sched, E, M, Y, N, K, src, weights, T,
+                                stream);
 }
 
 }  // extern "C"

@@ -453,6 +453,28 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched(const uint8_t* A, co
                                                             const void* sched, int E, int M, void* Y_bf16,
                                                             int N, int K, void* stream);
 
+/* gemm_nvfp4_w4a4_grouped_packed_sched with the top-1 combine fused into its
+ * epilogue. Page 2's MegaMoE does its combine inside the expert kernel; this is
+ * the same idea for one expert per token.
+ *   - Grouped row r (the row of token pair src[r] in expert order, as
+ *     nvfp4_moe_route / nvfp4_moe_permute_rows produce it with k = 1) is written
+ *     to Y_bf16 row src[r]: Y[src[r]][n] = BF16(gA*gW[e] * w * acc[r][n]).
+ *   - w is weights[src[r]] (device float [T]); w = 1 when weights is NULL.
+ *   - The result equals nvfp4_moe_combine over the unfused product's rows,
+ *     except that it is rounded to BF16 once instead of twice. The grouped
+ *     rows never reach memory.
+ *   - src: device int32 [M], a permutation of [0, T) in top-1 routing. Every
+ *     Y row named by src is written once; other rows of Y are left as they are.
+ *   - Y_bf16: device [T][N], caller-owned.
+ *   - M <= T; N even.
+ *   - A src entry outside [0, T) is not written. It makes the next
+ *     nvfp4_check_device_error return NVFP4_ERR_INVALID_ARG.
+ *   - Everything else as gemm_nvfp4_w4a4_grouped_packed_sched. */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched_combine(
+    const uint8_t* A, const uint8_t* sA_packed, const uint8_t* W, const uint8_t* sW_packed,
+    const void* sched, int E, int M, const int32_t* src, const float* weights, void* Y_bf16, int T,
+    int N, int K, void* stream);
+
 /* ---- diagnostics ----------------------------------------------------------- */
 
 /* Thread-local text of the last error returned on this host thread ("" if none). */

@@ -1,11 +1,13 @@
 """The grouped product planned on the device from device-resident expert offsets:
 the same bytes as the host-planned entry (same tiles, same alphas), parity with the
-oracle, bad offsets reported, and a whole MoE layer captured in one CUDA graph."""
+oracle, bad offsets reported, and a whole MoE layer captured in one CUDA graph; and
+the same product with the top-1 combine fused into its epilogue."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
+from oracle import moe as om
 import block_scaled_precision_nvfp4_b200 as nv
 from block_scaled_precision_nvfp4_b200 import workloads as wl
 
@@ -142,3 +144,79 @@ def test_whole_moe_layer_in_one_cuda_graph():
     nv.nvfp4_check_device_error()
     assert torch.equal(bufs["y"].view(torch.int16), eager.view(torch.int16))
     del g
+
+
+def _top1_layer(counts, N, K, seed):
+    """Tokens routed top-1 to experts with the given token counts, in a shuffled token
+    order; returns the inputs and the routed, permuted, packed state of the layer."""
+    rng = np.random.default_rng(seed)
+    E, T = len(counts), int(sum(counts))
+    ids = rng.permutation(np.repeat(np.arange(E, dtype=np.int32), counts)).reshape(T, 1)
+    A = wl.uniform_operand(rng, T, K)
+    Ws = [wl.uniform_operand(rng, N, K) for _ in counts]
+    Wc = np.stack([w.codes for w in Ws]); Wsc = np.stack([w.scales for w in Ws])
+    gW = rng.choice([0.25, 0.5, 1.0, 2.0], E)
+    w = rng.random(T).astype(np.float32) + np.float32(0.5)
+    off, dest, src = nv.moe_route(_dev(ids), E)
+    gc = nv.moe_permute_rows(_dev(A.codes), src, 1)
+    gs = nv.moe_permute_rows(_dev(A.scales), src, 1)
+    sw = nv.nvfp4_pack_scales_grouped(_dev(Wsc.reshape(E * N, K // 16)),
+                                      [e * N for e in range(E + 1)], K)
+    sched = nv.GroupedSchedule(off, E, T, N, K, gW, gA=1.5)
+    sa = sched.pack(gs)
+    return dict(E=E, T=T, ids=ids, A=A, Wc=Wc, Wsc=Wsc, gW=gW, w=w, off=off, dest=dest, src=src,
+                gc=gc, gs=gs, sw=sw, sched=sched, sa=sa, Wc_d=_dev(Wc))
+
+
+FUSED = [([300, 129, 0, 1, 256, 14], 264, 512), ([700], 512, 256), ([5, 60, 127, 128, 3], 256, 768),
+         ([40] * 9, 136, 256)]
+
+
+@pytest.mark.parametrize("counts,N,K", FUSED)
+def test_fused_top1_combine_against_the_oracle(counts, N, K):
+    """Y[t] = BF16(w[t] * alpha_e * sum_k ...) for each token t routed to expert e, rounded
+    once, against the oracle's grouped product and combine in FP64."""
+    L = _top1_layer(counts, N, K, sum(counts) + N)
+    y = L["sched"].gemm_combine(L["gc"], L["sa"], L["Wc_d"], L["sw"], L["src"], L["T"],
+                                weights=_dev(L["w"]))
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    ro, rd, rs = om.route(L["ids"], L["E"])
+    g = om.permute_rows(L["A"].codes, rs, 1), om.permute_rows(L["A"].scales, rs, 1)
+    Yg = oracle.gemm_grouped_w4a4(g[0], g[1], 1.5, L["Wc"], L["Wsc"], L["gW"], ro, N, K)
+    ref = om.combine(Yg, rd, L["w"].reshape(-1, 1), L["T"], 1)
+    check(bf16_to_f64(y), ref, f"fused combine {counts}")
+
+
+@pytest.mark.parametrize("counts,N,K", FUSED[:2])
+def test_fused_top1_combine_against_the_unfused_layer(counts, N, K):
+    L = _top1_layer(counts, N, K, 3 * sum(counts) + K)
+    s = L["sched"]
+    yg = s.gemm(L["gc"], L["sa"], L["Wc_d"], L["sw"])
+    # without weights the fused epilogue writes the unfused rows, permuted: same bits
+    y1 = s.gemm_combine(L["gc"], L["sa"], L["Wc_d"], L["sw"], L["src"], L["T"])
+    y0 = nv.moe_combine(yg, L["dest"], None, L["T"], 1)
+    # with weights the unfused path rounds twice, the fused one once
+    wd = _dev(L["w"])
+    y2 = s.gemm_combine(L["gc"], L["sa"], L["Wc_d"], L["sw"], L["src"], L["T"], weights=wd)
+    y3 = nv.moe_combine(yg, L["dest"], wd.reshape(-1, 1), L["T"], 1)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y0.view(torch.int16))
+    a, b = bf16_to_f64(y2), bf16_to_f64(y3)
+    assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)))
+
+
+def test_fused_combine_reports_a_bad_destination_and_skips_it():
+    L = _top1_layer([100, 28], 256, 256, 77)
+    T = L["T"]
+    src = L["src"].clone()
+    victim = int(src[5].item())
+    src[5] = T                                                    # outside [0, T)
+    y = torch.full((T, 256), 3.0, dtype=torch.bfloat16, device="cuda")
+    L["sched"].gemm_combine(L["gc"], L["sa"], L["Wc_d"], L["sw"], src, T, out=y)
+    with pytest.raises(nv.NvFp4Error) as e:
+        nv.nvfp4_check_device_error()
+    assert e.value.status == nv.Status.INVALID_ARG
+    assert bool((y[victim].float() == 3.0).all())                 # that token's row is not written
+    others = [int(t) for t in L["src"].tolist() if int(t) != victim]
+    assert not bool((y[others].float() == 3.0).all())
