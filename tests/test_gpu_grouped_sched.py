@@ -88,9 +88,11 @@ def test_bad_device_offsets_are_reported_and_write_nothing():
     assert bool((y.float() == 7.0).all())
 
 
-def test_whole_moe_layer_in_one_cuda_graph():
-    """quantise -> route -> permute -> schedule -> pack -> grouped W4A4 -> combine,
-    captured once and replayed, equals the eager layer bit for bit."""
+@pytest.mark.parametrize("fused", [False, True])
+def test_whole_moe_layer_in_one_cuda_graph(fused):
+    """quantise -> route -> permute -> schedule -> pack -> grouped W4A4 -> combine (a
+    separate kernel, or fused into the product's epilogue), captured once and
+    replayed, equals the eager layer bit for bit."""
     rng = np.random.default_rng(21)
     T, E, N, K = 700, 4, 384, 512
     x = torch.from_numpy(rng.standard_normal((T, K)).astype(np.float32)).to(torch.bfloat16).cuda()
@@ -124,8 +126,11 @@ def test_whole_moe_layer_in_one_cuda_graph():
         nv.moe_permute_rows(b["scales"], src, 1, out=b["gs"], stream=s)
         sched = nv.GroupedSchedule(off, E, T, N, K, gws, gA=b["g"][:1], stream=s)
         sched.pack(b["gs"], out=b["sa"], stream=s)
-        sched.gemm(b["gc"], b["sa"], Wc, sw, out=b["yg"], stream=s)
-        nv.moe_combine(b["yg"], dest, w, T, 1, out=b["y"], stream=s)
+        if fused:
+            sched.gemm_combine(b["gc"], b["sa"], Wc, sw, src, T, weights=w, out=b["y"], stream=s)
+        else:
+            sched.gemm(b["gc"], b["sa"], Wc, sw, out=b["yg"], stream=s)
+            nv.moe_combine(b["yg"], dest, w, T, 1, out=b["y"], stream=s)
         return sched, off, dest, src
 
     cur = torch.cuda.current_stream()
