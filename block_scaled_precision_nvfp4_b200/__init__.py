@@ -94,6 +94,7 @@ C_FUNCTIONS = {
     "nvfp4_pack_scales": (_I, [_P, _I, _I, _P, _P]),
     "gemm_nvfp4_w4a4_packed": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _P]),
     "nvfp4_w4a4_packed_workspace_bytes": (_Z, [_I, _I, _I, _I]),
+    "nvfp4_w4a4_packed_workspace_bytes_for": (_Z, [_I, _I, _I, _I, _I]),
     "gemm_nvfp4_w4a4_packed_ws": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _I, _P, _Z, _P]),
     "gemm_w4a16": (_I, [_P, _P, _P, _F, _P, _I, _I, _I, _P]),
     "gemm_nvfp4_w4a4_grouped": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),

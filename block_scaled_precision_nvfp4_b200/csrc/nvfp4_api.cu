@@ -650,12 +650,17 @@ nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* sA_packed, 
     return launch_w4a4_pair(A, sA_packed, gA, W, sW_packed, gW, Y, M, N, K, 0, nullptr, 0, stream);
 }
 
+size_t nvfp4_w4a4_packed_workspace_bytes_for(int M, int N, int K, int max_pairs, int num_sms) {
+    if (M <= 0 || N <= 0 || K <= 0 || max_pairs < 0 || num_sms < 2) return 0;
+    const PairPlan plan = pair_plan(M, N, K, num_sms, max_pairs, true);
+    return plan.slots > 0 ? nvfp4::w4a4_pair::split_workspace_bytes(plan.slots) : 0;
+}
+
 size_t nvfp4_w4a4_packed_workspace_bytes(int M, int N, int K, int max_pairs) {
     int dev;
     DevInfo info;
-    if (M <= 0 || N <= 0 || K <= 0 || max_pairs < 0 || !current_device(dev, info)) return 0;
-    const PairPlan plan = pair_plan(M, N, K, info.num_sms, max_pairs, true);
-    return plan.slots > 0 ? nvfp4::w4a4_pair::split_workspace_bytes(plan.slots) : 0;
+    if (!current_device(dev, info)) return 0;
+    return nvfp4_w4a4_packed_workspace_bytes_for(M, N, K, max_pairs, info.num_sms);
 }
 
 nvfp4_status gemm_nvfp4_w4a4_packed_ws(const uint8_t* A, const uint8_t* sA_packed, float gA,

@@ -252,6 +252,12 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a4_packed(const uint8_t* A, const uint8_t* s
  * about 38 MB on a 148-SM part.  0 also when the device cannot be queried. */
 NVFP4_API size_t nvfp4_w4a4_packed_workspace_bytes(int M, int N, int K, int max_pairs);
 
+/* The same for a device with `num_sms` SMs (148 on a B200), without querying any
+ * device: a pure function, usable with no GPU (for instance to size a workspace
+ * before a device is opened).  0 for num_sms < 2 or a non-positive size. */
+NVFP4_API size_t nvfp4_w4a4_packed_workspace_bytes_for(int M, int N, int K, int max_pairs,
+                                                       int num_sms);
+
 /* gemm_nvfp4_w4a4_packed with the last waves of tiles balanced over the pairs
  * (stream-K).  This is a design of this library, not of the pages; the product
  * is the page-1 module doc's NVFP4 row, as for gemm_nvfp4_w4a4_packed.

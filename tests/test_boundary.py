@@ -227,3 +227,40 @@ def test_node_exec_bad_formats_and_arguments():
     assert lib.nvfp4_node_exec(100, 0, None, a, 3, out) == nv.Status.INVALID_ARG
     assert lib.nvfp4_node_exec(100, 0, None, None, 0, None) == nv.Status.OK
     assert nv.nvfp4_node_exec(100, []) == []
+
+
+def test_stream_k_workspace_plan_needs_no_device():
+    """The pair kernel's tile balance plan (pure host arithmetic): a workspace only
+    when the last wave of 256 x 256 tiles would be at most 60 % full, 512 KB per pair
+    boundary plus 64 bytes of tickets each (rounded up to 256)."""
+    lib = nv.load_library()
+    f = lib.nvfp4_w4a4_packed_workspace_bytes_for
+
+    def need(pairs):
+        slots = pairs - 1
+        return (slots * 64 + 255) // 256 * 256 + slots * 2 * 2 * 8 * 32 * 128 * 4
+
+    # FFN down on 148 SMs: 336 tiles on 74 pairs, last wave 40/74 = 54 % full -> cut
+    assert f(4096, 5376, 14336, 0, 148) == need(74) == 38277888
+    # 6144 x 5376: 504 tiles, last wave 60/74 = 81 % full -> whole tiles
+    assert f(6144, 5376, 14336, 0, 148) == 0
+    # whole waves: 296 tiles on 74 pairs
+    assert f(2048, 9472, 14336, 0, 148) == 0
+    # fewer tiles than pairs: no full wave to balance against
+    assert f(1024, 1024, 14336, 0, 148) == 0
+    # a single K-block cannot be cut
+    assert f(4096, 5376, 256, 0, 148) == 0
+    # max_pairs caps the pairs: 12 tiles on 5 pairs (last wave 40 %), on 7 (71 %)
+    assert f(768, 1024, 1024, 5, 148) == need(5)
+    assert f(768, 1024, 1024, 7, 148) == 0
+    # the threshold is inclusive: 8 tiles on 5 pairs leave a 60 % full last wave
+    assert f(512, 1024, 1024, 5, 148) == need(5)
+    # fewer SMs, fewer pairs
+    assert f(4096, 5376, 14336, 0, 132) == need(66)     # 336 on 66: 6/66 full
+    # degenerate arguments
+    for args in [(0, 5376, 14336, 0, 148), (4096, 0, 14336, 0, 148), (4096, 5376, 0, 0, 148),
+                 (4096, 5376, 14336, -1, 148), (4096, 5376, 14336, 0, 1)]:
+        assert f(*args) == 0
+    # without a device the device query gives 0
+    assert lib.nvfp4_w4a4_packed_workspace_bytes(4096, 5376, 14336, 0) == 0 or \
+        __import__("torch").cuda.is_available()
