@@ -200,7 +200,10 @@ __device__ __forceinline__ bool combine_partial(float* __restrict__ ws, unsigned
         seen = __shfl_sync(0xffffffffu, seen, 0);
         if (seen == 0) return false;
     }
+    // lane 0 saw the other contributor's ticket (an acquire load, or the add followed
+    // by this fence); the warp barrier then orders every lane's reads after it
     __threadfence();
+    __syncwarp();
     const float4* other =
         reinterpret_cast<const float4*>(ws + part_offset(sg.slot, sg.side ^ 1, rank, w)) + lane;
 #pragma unroll
