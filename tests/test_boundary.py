@@ -264,3 +264,30 @@ def test_stream_k_workspace_plan_needs_no_device():
     # without a device the device query gives 0
     assert lib.nvfp4_w4a4_packed_workspace_bytes(4096, 5376, 14336, 0) == 0 or \
         __import__("torch").cuda.is_available()
+
+
+def test_balanced_w4a4_argument_errors_need_no_device():
+    lib = nv.load_library()
+
+    def call(A=16, M=512, N=512, K=1024, max_pairs=0, ws=None, nws=0):
+        return lib.gemm_nvfp4_w4a4_packed_ws(A, 16, 1.0, 16, 16, 1.0, 16, M, N, K, max_pairs, ws,
+                                             nws, None)
+    assert call(max_pairs=-1) == nv.Status.INVALID_ARG
+    assert call(M=-1) == nv.Status.INVALID_ARG
+    assert call(K=320) == nv.Status.INVALID_ARG              # the pair kernel needs K % 256
+    assert call(A=0) == nv.Status.INVALID_ARG
+    assert call(A=24) == nv.Status.MISALIGNED
+
+
+def test_fused_combine_argument_errors_need_no_device():
+    lib = nv.load_library()
+
+    def call(E=2, M=64, src=16, T=64, N=256, K=256):
+        return lib.gemm_nvfp4_w4a4_grouped_packed_sched_combine(16, 16, 16, 16, 16, E, M, src, None,
+                                                                16, T, N, K, None)
+    assert call(src=None) == nv.Status.INVALID_ARG           # rows but no destinations
+    assert call(M=65) == nv.Status.INVALID_ARG               # top-1: at most one row per token
+    assert call(T=-1) == nv.Status.INVALID_ARG
+    assert call(N=255) == nv.Status.INVALID_ARG              # rows leave as 4-byte pairs
+    assert call(E=0) == nv.Status.INVALID_ARG
+    assert call(K=320) == nv.Status.INVALID_ARG
