@@ -26,7 +26,8 @@ __all__ = [
     "nvfp4_kind_of", "nvfp4_exec_of", "nvfp4_exec_of_arch", "nvfp4_pair_name",
     "nvfp4_exec_name", "nvfp4_set_fp4_kernel_disabled", "nvfp4_version",
     "nvfp4_check_device_error", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8", "gemm_nvfp4_w4a8", "gemm_w4a16",
-    "gemm_nvfp4_w4a4_grouped", "nvfp4_scale_layout_bytes", "nvfp4_pack_scales",
+    "gemm_nvfp4_w4a4_grouped", "gemm_nvfp4_w4a4_grouped_host", "nvfp4_scale_layout_bytes",
+    "nvfp4_pack_scales", "nvfp4_prepare_scales", "nvfp4_workspace_size", "Op",
     "gemm_nvfp4_w4a4_packed", "nvfp4_w4a4_packed_workspace_bytes", "w4a4_packed_workspace",
     "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
     "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "nvfp4_fp4_fallback",
@@ -54,6 +55,18 @@ class Exec(enum.IntEnum):
     BF16_WIDEN = 2
     NO_FP4_KERNEL = 3
     NO_PATH = 4
+
+
+class Op(enum.IntEnum):
+    """Operations of nvfp4_workspace_size."""
+    W4A4 = 0
+    VIA_FP8 = 1
+    W4A16 = 2
+    W4A4_GROUPED = 3
+    W4A8 = 4
+    W4A4_PACKED = 5
+    QUANTIZE = 6
+    MOE_ROUTE = 7
 
 
 class Status(enum.IntEnum):
@@ -97,7 +110,10 @@ C_FUNCTIONS = {
     "nvfp4_w4a4_packed_workspace_bytes_for": (_Z, [_I, _I, _I, _I, _I]),
     "gemm_nvfp4_w4a4_packed_ws": (_I, [_P, _P, _F, _P, _P, _F, _P, _I, _I, _I, _I, _P, _Z, _P]),
     "gemm_w4a16": (_I, [_P, _P, _P, _F, _P, _I, _I, _I, _P]),
-    "gemm_nvfp4_w4a4_grouped": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
+    "gemm_nvfp4_w4a4_grouped": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _I, _I, _P, _Z, _P]),
+    "gemm_nvfp4_w4a4_grouped_host": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
+    "nvfp4_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "nvfp4_prepare_scales": (_I, [_P, _P, _I, _I, _P]),
     "nvfp4_grouped_scale_layout_bytes": (_Z, [_P, _I, _I]),
     "nvfp4_pack_scales_grouped": (_I, [_P, _P, _I, _I, _P, _P]),
     "gemm_nvfp4_w4a4_grouped_packed": (_I, [_P, _P, _F, _P, _P, _P, _P, _I, _P, _I, _I, _P]),
@@ -408,8 +424,43 @@ def gemm_w4a16(A, W, sW, gW, out=None, stream=None):
     return out
 
 
-def gemm_nvfp4_w4a4_grouped(A, sA, gA, W, sW, gW, offsets, out=None, stream=None):
-    """Grouped W4A4: W [E,N,K/2], sW [E,N,K/16], gW (E floats), offsets (E+1 ints, host)."""
+def gemm_nvfp4_w4a4_grouped(A, sA, gA, W, sW, gW, offsets, out=None, workspace=None,
+                            stream=None):
+    """Grouped W4A4: W [E,N,K/2], sW [E,N,K/16], gW (E floats).  With offsets a CUDA
+    int32 tensor [E+1], the C entry gemm_nvfp4_w4a4_grouped (device offsets, the
+    plan made on the device; `workspace` a CUDA uint8 tensor of at least
+    nvfp4_workspace_size(Op.W4A4_GROUPED, M, N, K, E) bytes, allocated here if None);
+    with host offsets (E+1 ints), gemm_nvfp4_w4a4_grouped_host."""
+    torch = _torch()
+    if not (isinstance(offsets, torch.Tensor) and offsets.is_cuda):
+        return gemm_nvfp4_w4a4_grouped_host(A, sA, gA, W, sW, gW, offsets, out, stream)
+    M, half_k = A.shape
+    K = 2 * half_k
+    E, N = W.shape[0], W.shape[1]
+    pa = _dev_tensor(A, torch.uint8, (M, K // 2), "A")
+    psa = _dev_tensor(sA, torch.uint8, (M, K // 16), "sA")
+    pw = _dev_tensor(W, torch.uint8, (E, N, K // 2), "W")
+    psw = _dev_tensor(sW, torch.uint8, (E, N, K // 16), "sW")
+    po = _dev_tensor(offsets, torch.int32, (E + 1,), "offsets")
+    gws = (ctypes.c_float * E)(*[float(x) for x in gW])
+    need = int(load_library().nvfp4_workspace_size(int(Op.W4A4_GROUPED), M, N, K, E))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=A.device)
+    if workspace.dtype != torch.uint8 or not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
+    _err(load_library().gemm_nvfp4_w4a4_grouped(pa, psa, float(gA), pw, psw,
+                                                ctypes.cast(gws, ctypes.c_void_p), po, E, M, py,
+                                                N, K, workspace.data_ptr(), workspace.numel(),
+                                                _stream_ptr(stream)))
+    return out
+
+
+def gemm_nvfp4_w4a4_grouped_host(A, sA, gA, W, sW, gW, offsets, out=None, stream=None):
+    """Grouped W4A4 planned on the host: W [E,N,K/2], sW [E,N,K/16], gW (E floats),
+    offsets (E+1 ints, host)."""
     torch = _torch()
     M, half_k = A.shape
     K = 2 * half_k
@@ -425,10 +476,31 @@ def gemm_nvfp4_w4a4_grouped(A, sA, gA, W, sW, gW, offsets, out=None, stream=None
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     py = _dev_tensor(out, torch.bfloat16, (M, N), "out")
-    _err(load_library().gemm_nvfp4_w4a4_grouped(pa, psa, float(gA), pw, psw,
-                                                ctypes.cast(gws, ctypes.c_void_p),
-                                                ctypes.cast(off, ctypes.c_void_p), E, py, N, K,
-                                                _stream_ptr(stream)))
+    _err(load_library().gemm_nvfp4_w4a4_grouped_host(pa, psa, float(gA), pw, psw,
+                                                     ctypes.cast(gws, ctypes.c_void_p),
+                                                     ctypes.cast(off, ctypes.c_void_p), E, py, N,
+                                                     K, _stream_ptr(stream)))
+    return out
+
+
+def nvfp4_workspace_size(op, M, N, K, E=1) -> int:
+    """Device bytes of caller workspace operation `op` (an Op) needs."""
+    return int(load_library().nvfp4_workspace_size(int(op), int(M), int(N), int(K), int(E)))
+
+
+def nvfp4_prepare_scales(s, K=None, out=None, stream=None):
+    """Plain scales uint8 [rows, K/16] -> the MMA scale layout (uint8 1-D), through the C
+    entry nvfp4_prepare_scales."""
+    torch = _torch()
+    rows, groups = s.shape
+    K = 16 * groups if K is None else int(K)
+    ps = _dev_tensor(s, torch.uint8, (rows, K // 16), "s")
+    n = nvfp4_scale_layout_bytes(rows, K)
+    if out is None:
+        out = torch.empty(max(n, 16), dtype=torch.uint8, device=s.device)
+    if out.dtype != torch.uint8 or not out.is_cuda or out.numel() < n or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous CUDA uint8 tensor of >= {n} bytes")
+    _err(load_library().nvfp4_prepare_scales(ps, out.data_ptr(), rows, K, _stream_ptr(stream)))
     return out
 
 
@@ -565,13 +637,19 @@ class GroupedSchedule:
     gemm(A, sA_packed, W, sW_packed) -> Y, with no host round trip."""
 
     def __init__(self, offsets, E, M, N, K, gW, gA=1.0, stream=None):
-        import ctypes
         torch = _torch()
         self.E, self.M, self.N, self.K = int(E), int(M), int(N), int(K)
+        self.buf = torch.empty(int(load_library().nvfp4_grouped_sched_bytes()),
+                               dtype=torch.uint8, device=offsets.device)
+        self.plan(offsets, gW, gA, stream)
+
+    def plan(self, offsets, gW, gA=1.0, stream=None):
+        """(Re)plans into this schedule's buffer from new device offsets (same E, M,
+        N, K); later pack/gemm calls on the stream use the new plan."""
+        import ctypes
+        torch = _torch()
         lib = load_library()
         po = _dev_tensor(offsets, torch.int32, (self.E + 1,), "offsets")
-        self.buf = torch.empty(int(lib.nvfp4_grouped_sched_bytes()), dtype=torch.uint8,
-                               device=offsets.device)
         gws = (ctypes.c_float * self.E)(*[float(x) for x in gW])
         ga_dev, ga = None, 1.0
         if isinstance(gA, torch.Tensor):

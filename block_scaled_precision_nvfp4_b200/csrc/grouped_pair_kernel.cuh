@@ -219,10 +219,6 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const int cid = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
-    const int N = p.N, K = p.K;
-    const int tiles = p.tile_start[p.E];
-    const int num_kb = K / BK;
-    const int wblocks = (N + 127) / 128;  // packed 128-row blocks of one expert's sW
     volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
@@ -245,8 +241,13 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     // the set-up above overlaps the kernel before this one (scale packing or the
-    // schedule, when launched programmatically); their output is read only from here
+    // schedule, when launched programmatically); their output -- the packed scales
+    // and, with p_dev, the schedule itself -- is read only from here
     grid_dependency_wait();
+    const int N = p.N, K = p.K;
+    const int tiles = p.tile_start[p.E];
+    const int num_kb = K / BK;
+    const int wblocks = (N + 127) / 128;  // packed 128-row blocks of one expert's sW
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)

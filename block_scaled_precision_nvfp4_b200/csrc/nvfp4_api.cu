@@ -501,32 +501,24 @@ nvfp4_status nvfp4_quantize_bf16(const void* X, int rows, int K, uint8_t* codes,
 // device scratch.  This variant keeps them in a static device array instead, so
 // a caller that cannot allocate device memory (or cannot keep a scratch buffer
 // between calls) can still quantise.  The array lives in every GPU that loads
-// the library until the process exits; its device address is looked up once
-// per device.
+// the library until the process exits.
 namespace {
 constexpr size_t kNoAllocScratchBytes = 256;  // the stated maximum; the quantiser needs 16
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 static_assert(NVFP4_QUANTIZE_WORKSPACE_BYTES <= kNoAllocScratchBytes,
               "the static scratch must hold the quantiser's workspace");
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kMaxDevices] = {};
-
-// The device address of g_noalloc_scratch on the current device (the host-side
-// name is only a stand-in for it), looked up on the first call per device.
-nvfp4_status noalloc_scratch(int dev, void** out) {
-    if (dev < 0 || dev >= kMaxDevices)
-        return fail(NVFP4_ERR_CUDA, "device %d is beyond the %d devices this entry point tracks", dev,
-                    kMaxDevices);
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_addr[dev]) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "looking up the static quantiser scratch");
-        g_noalloc_addr[dev] = p;
-    }
-    *out = g_noalloc_addr[dev];
+// The device address of g_noalloc_scratch in the current context (the host-side
+// name is only a stand-in for it).  Looked up on every call: the address belongs
+// to a context, not to a device ordinal, so a cached one could outlive its context
+// (after cudaDeviceReset, or under a caller's own driver context).  The lookup
+// allocates nothing; the first one in a context loads the library's device code
+// there, which is why the first call should come before any stream capture.
+nvfp4_status noalloc_scratch(void** out) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "looking up the static quantiser scratch");
+    *out = p;
     return NVFP4_OK;
 }
 }  // namespace
@@ -539,13 +531,8 @@ nvfp4_status nvfp4_quantize_bf16_noalloc(const void* X, int rows, int K, uint8_t
         return fail(NVFP4_ERR_INVALID_ARG,
                     "this call needs %zu bytes of scratch, more than the %zu of the static array",
                     need, kNoAllocScratchBytes);
-    int dev;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
-        cudaGetLastError();
-        return fail(NVFP4_ERR_CUDA, "cannot query the current CUDA device");
-    }
     void* scratch = nullptr;
-    nvfp4_status st = noalloc_scratch(dev, &scratch);
+    nvfp4_status st = noalloc_scratch(&scratch);
     if (st != NVFP4_OK) return st;
     return nvfp4_quantize_bf16(X, rows, K, codes, scales, scales_packed, g_out, scratch,
                                kNoAllocScratchBytes, stream);
@@ -905,10 +892,10 @@ nvfp4_status gemm_w4a16(const void* A, const uint8_t* W, const uint8_t* sW, floa
 }
 
 // ------------------------------------------------------------------------- grouped W4A4
-nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t* A, const uint8_t* sA, float gA,
-                                     const uint8_t* W, const uint8_t* sW, const float* gW_host,
-                                     const int32_t* offsets_host, int E, void* Y, int N, int K,
-                                     void* stream) {
+nvfp4_status gemm_nvfp4_w4a4_grouped_host(const uint8_t* A, const uint8_t* sA, float gA,
+                                          const uint8_t* W, const uint8_t* sW,
+                                          const float* gW_host, const int32_t* offsets_host, int E,
+                                          void* Y, int N, int K, void* stream) {
     namespace gk = nvfp4::grouped;
     if (E < 1 || E > gk::MAX_EXPERTS)
         return fail(NVFP4_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", gk::MAX_EXPERTS, E);
@@ -1237,6 +1224,96 @@ nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched_combine(const uint8_t* A,
     if (N % 2 != 0) return fail(NVFP4_ERR_INVALID_ARG, "the fused combine needs an even N (got %d)", N);
     return launch_grouped_sched(A, sA_packed, W, sW_packed, sched, E, M, Y, N, K, src, weights, T,
                                 stream);
+}
+
+
+// ------------------------------------------------------------------------- grouped W4A4 from plain
+// scales and device offsets: schedule, pack both scale matrices, product
+namespace {
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+// Offsets of the three parts of the grouped entry's workspace.
+struct GroupedWs {
+    size_t sched = 0, sa = 0, sw = 0, total = 0;
+};
+bool grouped_ws_layout(int M, int N, int K, int E, GroupedWs& w) {
+    if (M < 0 || N < 1 || E < 1 || E > nvfp4::grouped_pair::MAX_EXPERTS || K < 256 || K % 256 != 0)
+        return false;
+    w.sched = 0;
+    w.sa = round256(nvfp4_grouped_sched_bytes());
+    w.sw = w.sa + round256(nvfp4_grouped_scale_layout_bytes_bound(M, E, K));
+    w.total = w.sw + round256((size_t)E * (size_t)((N + 127) / 128) * 128 * (size_t)(K / 16));
+    return true;
+}
+}  // namespace
+
+nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t* A, const uint8_t* sA, float gA,
+                                     const uint8_t* W, const uint8_t* sW, const float* gW_host,
+                                     const int32_t* offsets_dev, int E, int total_M, void* Y,
+                                     int N, int K, void* workspace, size_t ws_bytes,
+                                     void* stream) {
+    namespace gp = nvfp4::grouped_pair;
+    if (E < 1 || E > gp::MAX_EXPERTS)
+        return fail(NVFP4_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", gp::MAX_EXPERTS, E);
+    nvfp4_status st = check_w4a4_args(A, sA, W, sW, Y, total_M, N, K);
+    if (st != NVFP4_OK) return st;
+    if (K % gp::BK != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "the grouped path needs K %% 256 == 0 (got %d)", K);
+    if ((int64_t)E * N > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "E*N too large");
+    if (!offsets_dev || !gW_host) return fail(NVFP4_ERR_INVALID_ARG, "null offsets or gW");
+    GroupedWs w;
+    if (!grouped_ws_layout(total_M, N, K, E, w)) return fail(NVFP4_ERR_INVALID_ARG, "bad sizes");
+    if (total_M == 0 || N == 0) return ok();
+    if (!workspace || ws_bytes < w.total)
+        return fail(NVFP4_ERR_INVALID_ARG,
+                    "the workspace must hold nvfp4_workspace_size(NVFP4_OP_W4A4_GROUPED, ...) = %zu "
+                    "bytes (got %zu)", w.total, ws_bytes);
+    if (!aligned16(workspace)) return fail(NVFP4_ERR_MISALIGNED, "the workspace must be 16-byte aligned");
+    int dev;
+    DevInfo info;
+    if ((st = check_fp4_path(dev, info)) != NVFP4_OK) return st;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    void* sched = ws + w.sched;
+    uint8_t* sa_packed = ws + w.sa;
+    uint8_t* sw_packed = ws + w.sw;
+    // the weights' groups: E experts of N rows each
+    int32_t woff[nvfp4::grouped_pair::MAX_EXPERTS + 1];
+    for (int e = 0; e <= E; ++e) woff[e] = e * N;
+    if ((st = nvfp4_grouped_schedule(offsets_dev, E, total_M, N, K, nullptr, gA, gW_host, sched,
+                                     stream)) != NVFP4_OK)
+        return st;
+    if ((st = nvfp4_pack_scales_grouped_sched(sA, total_M, E, K, sched, sa_packed, stream)) != NVFP4_OK)
+        return st;
+    if ((st = nvfp4_pack_scales_grouped(sW, woff, E, K, sw_packed, stream)) != NVFP4_OK) return st;
+    return launch_grouped_sched(A, sa_packed, W, sw_packed, sched, E, total_M, Y, N, K, nullptr,
+                                nullptr, 0, stream);
+}
+
+// ------------------------------------------------------------------------- generic queries
+size_t nvfp4_workspace_size(int op, int M, int N, int K, int E) {
+    switch (op) {
+        case NVFP4_OP_W4A4:
+        case NVFP4_OP_VIA_FP8:
+        case NVFP4_OP_W4A16:
+        case NVFP4_OP_W4A8:
+            return 0;
+        case NVFP4_OP_W4A4_GROUPED: {
+            GroupedWs w;
+            return grouped_ws_layout(M, N, K, E, w) ? w.total : 0;
+        }
+        case NVFP4_OP_W4A4_PACKED:
+            return nvfp4_w4a4_packed_workspace_bytes(M, N, K, 0);
+        case NVFP4_OP_QUANTIZE:
+            return nvfp4_quantize_workspace_bytes();
+        case NVFP4_OP_MOE_ROUTE:
+            return nvfp4_moe_route_workspace_bytes(M, E);
+        default:
+            return SIZE_MAX;
+    }
+}
+
+nvfp4_status nvfp4_prepare_scales(const uint8_t* s_plain, uint8_t* s_mma, int rows, int K,
+                                  void* stream) {
+    return nvfp4_pack_scales(s_plain, rows, K, s_mma, stream);
 }
 
 }  // extern "C"

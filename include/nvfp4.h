@@ -149,9 +149,12 @@ NVFP4_API const char* nvfp4_exec_name(nvfp4_exec e);
 
 /* ---- matmuls --------------------------------------------------------------- */
 
-/* W4A4 on the block-scaled FP4 MMA (tcgen05.mma kind::mxf4nvf4, scale_vec::4X,
- * E4M3 scales, FP32 accumulation in tensor memory, fused alpha and BF16
- * epilogue).  M, N >= 0 (0 returns OK and does nothing); K >= 32, K % 32 == 0.
+/* W4A4 on the block-scaled FP4 MMA (metrale_circuit `hardware::exec` module
+ * doc, bullet 1, the NVFP4 row: NVFP4 activations take the block-scaled FP4
+ * MMA; the product is the operation at the top of this file).  tcgen05.mma
+ * kind::mxf4nvf4, scale_vec::4X, E4M3 scales, FP32 accumulation in tensor
+ * memory, fused alpha and BF16 epilogue; plain [rows][K/16] scales, rearranged
+ * on chip.  M, N >= 0 (0 returns OK and does nothing); K >= 32, K % 32 == 0.
  * Requires exec_of(device, NVFP4, NVFP4) == FP4_MMA, else NVFP4_ERR_NO_FP4_KERNEL
  * or NVFP4_ERR_NOPATH. */
 NVFP4_API nvfp4_status gemm_nvfp4_w4a4(const uint8_t* A, const uint8_t* sA, float gA,
@@ -235,7 +238,8 @@ NVFP4_API nvfp4_status nvfp4_quantize_bf16_noalloc(const void* X_bf16, int rows,
                                                    void* stream);
 
 /* gemm_nvfp4_w4a4 with both scale matrices already packed
- * (nvfp4_pack_scales).  Runs on pairs of SMs (tcgen05 cta_group::2, 256 x 256
+ * (nvfp4_pack_scales / nvfp4_prepare_scales); the same product, module doc
+ * bullet 1, the NVFP4 row.  Runs on pairs of SMs (tcgen05 cta_group::2, 256 x 256
  * tiles) and moves the packed scales with plain TMA tile loads, so no scale
  * rewrite happens inside the product.  Same operation, operands and errors as
  * gemm_nvfp4_w4a4, with K % 256 == 0. */
@@ -362,7 +366,11 @@ NVFP4_API nvfp4_status nvfp4_moe_combine(const void* Yg_bf16, int num_pairs, con
                                          const float* weights, int T, int k, int N, void* Y_bf16,
                                          void* stream);
 
-/* W4A16: BF16 activations A_bf16 [M][K] (row-major) times NVFP4 weights, the
+/* W4A16 (metrale_circuit `hardware::exec` module doc, bullet 1, the BF16 row:
+ * BF16 activations take the BF16 MMA, with any weight format widened in
+ * registers):
+ *     Y[m,n] = BF16( gW * sum_g sW[n,g] * sum_{k in g} a[m,k]*w[n,k] )
+ * BF16 activations A_bf16 [M][K] (row-major) times NVFP4 weights, the
  * weights widened to BF16 in registers (exactly: an E2M1 value times an E4M3
  * scale has at most 6 significant bits), FP32 accumulation, gW applied in the
  * epilogue, BF16 output Y [M][N].  Built for the memory-bound decode shape:
@@ -374,17 +382,49 @@ NVFP4_API nvfp4_status nvfp4_moe_combine(const void* Yg_bf16, int num_pairs, con
 NVFP4_API nvfp4_status gemm_w4a16(const void* A_bf16, const uint8_t* W, const uint8_t* sW, float gW,
                         void* Y_bf16, int M, int N, int K, void* stream);
 
-/* Grouped (MoE) W4A4: expert e owns rows offsets[e] .. offsets[e+1]-1 of A
- * (tokens grouped by expert), its weights W + e*N*K/2 ([N][K/2]), scales
- * sW + e*N*K/16 ([N][K/16]) and FP32 scale gW_host[e].  Y is [offsets[E]][N].
- * `offsets_host` (int32 [E+1], host memory, offsets[0] == 0, non-decreasing)
- * is read during the call only.  Experts with fewer than 128 rows run with
- * the operands swapped (Y_e^T = W_e . A_e^T: weight rows on the MMA's M side,
- * tokens on its N side).  1 <= E <= 256; K % 256 == 0. */
+/* Grouped (MoE) W4A4 with the expert offsets in device memory (page 2, the
+ * FlashInfer swapab_cutedsl_megakernel skill doc, Layout: the MoE kernel with
+ * swapped A/B operands for small per-expert M; each expert's product is the
+ * NVFP4 row of page 1's module doc, bullet 1).  Expert e owns rows
+ * offsets[e] .. offsets[e+1]-1 of A (tokens grouped by expert), its weights
+ * W + e*N*K/2 ([N][K/2]), plain scales sW + e*N*K/16 ([N][K/16]) and FP32
+ * scale gW_host[e]; Y is [total_M][N]:
+ *     Y[r,n] = BF16( gA*gW[e] * sum_g sA[r,g]*sW_e[n,g] * sum_{k in g} a[r,k]*w_e[n,k] )
+ *   offsets_dev  device int32 [E+1]: offsets[0] = 0, non-decreasing,
+ *                offsets[E] = total_M (for example nvfp4_moe_route's output);
+ *                never read on the host, so no round trip.  Offsets that break
+ *                these rules make the product write nothing and the next
+ *                nvfp4_check_device_error return NVFP4_ERR_INVALID_ARG.
+ *   gW_host      host float [E], read during the call only.
+ *   workspace    device memory, 16-byte aligned, caller-owned, of ws_bytes >=
+ *                nvfp4_workspace_size(NVFP4_OP_W4A4_GROUPED, total_M, N, K, E)
+ *                bytes (smaller is NVFP4_ERR_INVALID_ARG); needs no
+ *                initialisation; calls that overlap on the GPU need one each.
+ * The call plans the tiles on the device, packs both scale matrices into the
+ * workspace and runs the SM-pair product of gemm_nvfp4_w4a4_grouped_packed_sched:
+ * 256-token blocks of an expert as 256 x 256 tiles, an expert's last 1..128
+ * tokens swapped (weight rows on the MMA's M side, tokens on its N side).
+ * 1 <= E <= 256; N >= 1; K % 256 == 0; total_M == 0 returns OK and does
+ * nothing.  Callers that keep the weights' scales packed should call the
+ * _packed_sched entry points directly and skip the per-call weight packing. */
 NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped(const uint8_t* A, const uint8_t* sA, float gA,
                                      const uint8_t* W, const uint8_t* sW,
-                                     const float* gW_host, const int32_t* offsets_host,
-                                     int E, void* Y_bf16, int N, int K, void* stream);
+                                     const float* gW_host, const int32_t* offsets_dev,
+                                     int E, int total_M, void* Y_bf16, int N, int K,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
+/* The grouped product planned on the host from host offsets, on single SMs
+ * from plain scales (the same passages as gemm_nvfp4_w4a4_grouped).  Expert e
+ * owns rows offsets[e] .. offsets[e+1]-1 of A, W + e*N*K/2, sW + e*N*K/16 and
+ * gW_host[e]; Y is [offsets[E]][N].  `offsets_host` (int32 [E+1], host memory,
+ * offsets[0] == 0, non-decreasing) is read during the call only.  Blocks of
+ * fewer than 128 rows run with the operands swapped (Y_e^T = W_e . A_e^T:
+ * weight rows on the MMA's M side, tokens on its N side).  No workspace.
+ * 1 <= E <= 256; K % 256 == 0. */
+NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_host(const uint8_t* A, const uint8_t* sA, float gA,
+                                          const uint8_t* W, const uint8_t* sW,
+                                          const float* gW_host, const int32_t* offsets_host,
+                                          int E, void* Y_bf16, int N, int K, void* stream);
 
 /* Bytes of a grouped packed scale buffer: groups g = 0..E-1 own rows
  * offsets[g] .. offsets[g+1]-1 and each starts on a 128-row block, so the size
@@ -399,17 +439,18 @@ NVFP4_API size_t nvfp4_grouped_scale_layout_bytes(const int32_t* offsets_host, i
  * of tokens grouped by expert are packed this way per product; the weight
  * scales of E experts of N rows each are packed once with offsets
  * {0, N, 2N, ..., E*N}.  1 <= E <= 256, K % 64 == 0; the offsets rules of
- * gemm_nvfp4_w4a4_grouped.  Asynchronous on `stream`. */
+ * gemm_nvfp4_w4a4_grouped_host.  Asynchronous on `stream`. */
 NVFP4_API nvfp4_status nvfp4_pack_scales_grouped(const uint8_t* s_plain, const int32_t* offsets_host,
                                                  int E, int K, uint8_t* s_packed, void* stream);
 
-/* gemm_nvfp4_w4a4_grouped with packed scales: sA_packed packed by
- * nvfp4_pack_scales_grouped with these offsets, sW_packed with offsets
- * {0, N, ..., E*N}.  Runs on pairs of SMs (tcgen05 cta_group::2): 256-token
- * blocks of an expert as M = 256, N = 256 tiles; an expert's last 1..128
- * tokens (all of a small expert) swapped, 256 weight rows on the MMA's M side
- * and 128 token slots on its N side.  Same operation, operands and errors as
- * gemm_nvfp4_w4a4_grouped (K % 256 == 0). */
+/* gemm_nvfp4_w4a4_grouped_host with packed scales (page 2, swapab_cutedsl_megakernel,
+ * Layout: swap-AB for small M; page 1 module doc bullet 1, the NVFP4 row, per
+ * expert): sA_packed packed by nvfp4_pack_scales_grouped with these offsets,
+ * sW_packed with offsets {0, N, ..., E*N}.  Runs on pairs of SMs (tcgen05
+ * cta_group::2): 256-token blocks of an expert as M = 256, N = 256 tiles; an
+ * expert's last 1..128 tokens (all of a small expert) swapped, 256 weight rows
+ * on the MMA's M side and 128 token slots on its N side.  Same operation,
+ * operands and errors as gemm_nvfp4_w4a4_grouped_host (K % 256 == 0). */
 NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_packed(const uint8_t* A, const uint8_t* sA_packed,
                                                       float gA, const uint8_t* W,
                                                       const uint8_t* sW_packed,
@@ -417,9 +458,10 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_packed(const uint8_t* A, const ui
                                                       const int32_t* offsets_host, int E,
                                                       void* Y_bf16, int N, int K, void* stream);
 
-/* ---- grouped product with device-resident expert offsets -----------------
- * The grouped entry points above plan their tiles on the host from host
- * offsets.  These take offsets[E+1] in device memory (for example from
+/* ---- grouped product with device-resident expert offsets, packed scales ----
+ * (page 2, swapab_cutedsl_megakernel, Layout; page 1 module doc bullet 1, the
+ * NVFP4 row, per expert.)  The _host and _packed entry points above plan their
+ * tiles on the host from host offsets.  These take offsets[E+1] in device memory (for example from
  * nvfp4_moe_route), so a whole MoE layer runs with no host round trip and can
  * be captured in a CUDA graph: nvfp4_grouped_schedule plans on the device into
  * a small caller buffer, which the packing and the product then read.  Same
@@ -480,6 +522,36 @@ NVFP4_API nvfp4_status gemm_nvfp4_w4a4_grouped_packed_sched_combine(
     const uint8_t* A, const uint8_t* sA_packed, const uint8_t* W, const uint8_t* sW_packed,
     const void* sched, int E, int M, const int32_t* src, const float* weights, void* Y_bf16, int T,
     int N, int K, void* stream);
+
+/* ---- generic workspace query and scale preparation ------------------------ */
+
+/* The operations whose workspace nvfp4_workspace_size reports. */
+typedef enum {
+    NVFP4_OP_W4A4 = 0,          /* gemm_nvfp4_w4a4: none */
+    NVFP4_OP_VIA_FP8 = 1,       /* gemm_nvfp4_via_fp8: none */
+    NVFP4_OP_W4A16 = 2,         /* gemm_w4a16: none */
+    NVFP4_OP_W4A4_GROUPED = 3,  /* gemm_nvfp4_w4a4_grouped (M = total_M) */
+    NVFP4_OP_W4A8 = 4,          /* gemm_nvfp4_w4a8: none */
+    NVFP4_OP_W4A4_PACKED = 5,   /* gemm_nvfp4_w4a4_packed_ws on the current device, all pairs */
+    NVFP4_OP_QUANTIZE = 6,      /* nvfp4_quantize_bf16 (a constant) */
+    NVFP4_OP_MOE_ROUTE = 7      /* nvfp4_moe_route with num_pairs = M */
+} nvfp4_op;
+
+/* Device bytes of caller workspace that operation `op` (an nvfp4_op) needs for
+ * an M x N x K product over E experts (E is ignored by ungrouped ops).  0 when
+ * the call needs none or a size is invalid; SIZE_MAX for an unknown op.  Every
+ * workspace-taking entry point accepts a buffer of at least this size; none
+ * allocates device memory itself.  Host only (NVFP4_OP_W4A4_PACKED queries the
+ * current device's SM count and is 0 without a device). */
+NVFP4_API size_t nvfp4_workspace_size(int op, int M, int N, int K, int E);
+
+/* Plain E4M3 group scales s_plain [rows][K/16] -> the block-scaled MMA's scale
+ * layout in s_mma (nvfp4_scale_layout_bytes(rows, K) bytes): the same
+ * rearrangement as nvfp4_pack_scales (whose comment gives the layout), with the
+ * argument order of a prepare step.  K % 64 == 0; device pointers, 16-byte
+ * aligned, caller-owned; asynchronous on `stream`. */
+NVFP4_API nvfp4_status nvfp4_prepare_scales(const uint8_t* s_plain, uint8_t* s_mma, int rows, int K,
+                                            void* stream);
 
 /* ---- diagnostics ----------------------------------------------------------- */
 

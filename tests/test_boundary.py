@@ -112,8 +112,9 @@ def test_grouped_argument_errors_need_no_device():
     gws = (ctypes.c_float * 3)(1.0, 1.0, 1.0)
     def call(offs, E=2, K=256, N=64, A=16):
         o = (ctypes.c_int32 * len(offs))(*offs)
-        return lib.gemm_nvfp4_w4a4_grouped(A, 16, 1.0, 16, 16, ctypes.cast(gws, ctypes.c_void_p),
-                                           ctypes.cast(o, ctypes.c_void_p), E, 16, N, K, None)
+        return lib.gemm_nvfp4_w4a4_grouped_host(A, 16, 1.0, 16, 16,
+                                                ctypes.cast(gws, ctypes.c_void_p),
+                                                ctypes.cast(o, ctypes.c_void_p), E, 16, N, K, None)
     assert call([0, 6, 5]) == nv.Status.INVALID_ARG          # decreasing
     assert call([1, 6, 8]) == nv.Status.INVALID_ARG          # offsets[0] != 0
     assert call([0, 0], E=0) == nv.Status.INVALID_ARG        # no experts
@@ -291,3 +292,73 @@ def test_fused_combine_argument_errors_need_no_device():
     assert call(N=255) == nv.Status.INVALID_ARG              # rows leave as 4-byte pairs
     assert call(E=0) == nv.Status.INVALID_ARG
     assert call(K=320) == nv.Status.INVALID_ARG
+
+
+# The boundary's generic names: every call the hot-path scope lists exists under its
+# own name, with its own argument order.
+BOUNDARY_NAMES = ["nvfp4_exec_of", "nvfp4_pair_name", "gemm_nvfp4_w4a4", "gemm_nvfp4_via_fp8",
+                  "gemm_w4a16", "gemm_nvfp4_w4a4_grouped", "nvfp4_workspace_size",
+                  "nvfp4_prepare_scales", "nvfp4_last_error", "nvfp4_check_device_error"]
+
+
+def test_boundary_names_are_exported():
+    lib = nv.load_library()
+    declared = set(declared_functions())
+    for name in BOUNDARY_NAMES:
+        assert name in declared, name
+        assert hasattr(lib, name), name
+
+
+def test_workspace_size_per_op():
+    lib = nv.load_library()
+    Op = nv.Op
+    for op in (Op.W4A4, Op.VIA_FP8, Op.W4A16, Op.W4A8):
+        assert lib.nvfp4_workspace_size(int(op), 4096, 5376, 14336, 1) == 0
+    assert lib.nvfp4_workspace_size(int(Op.QUANTIZE), 4096, 0, 14336, 1) == \
+        lib.nvfp4_quantize_workspace_bytes()
+    assert lib.nvfp4_workspace_size(int(Op.MOE_ROUTE), 8192, 0, 0, 8) == \
+        lib.nvfp4_moe_route_workspace_bytes(8192, 8)
+    # grouped: the schedule, the packed activation scales (their bound) and the
+    # experts' packed weight scales, each rounded up to 256 bytes
+    M, N, K, E = 8192, 14336, 4096, 8
+    r = lambda b: (b + 255) // 256 * 256
+    expect = (r(lib.nvfp4_grouped_sched_bytes()) + r(lib.nvfp4_grouped_scale_layout_bytes_bound(M, E, K))
+              + r(E * ((N + 127) // 128) * 128 * (K // 16)))
+    assert lib.nvfp4_workspace_size(int(Op.W4A4_GROUPED), M, N, K, E) == expect
+    assert lib.nvfp4_workspace_size(int(Op.W4A4_GROUPED), M, N, 4000, E) == 0   # K % 256
+    assert lib.nvfp4_workspace_size(int(Op.W4A4_GROUPED), M, N, K, 0) == 0      # no experts
+    assert lib.nvfp4_workspace_size(99, 1, 1, 64, 1) == 2 ** 64 - 1             # unknown op
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.nvfp4_workspace_size(int(Op.W4A4_PACKED), 4096, 5376, 14336, 1) == 0
+
+
+def test_device_offset_grouped_argument_errors_need_no_device():
+    lib = nv.load_library()
+    gws = (ctypes.c_float * 2)(1.0, 1.0)
+    need = lib.nvfp4_workspace_size(int(nv.Op.W4A4_GROUPED), 64, 256, 256, 2)
+    assert need > 0
+
+    def call(E=2, M=64, N=256, K=256, A=16, off=16, ws=4096, ws_bytes=None):
+        return lib.gemm_nvfp4_w4a4_grouped(A, 16, 1.0, 16, 16, ctypes.cast(gws, ctypes.c_void_p),
+                                           off, E, M, 16, N, K, ws,
+                                           need if ws_bytes is None else ws_bytes, None)
+    assert call(E=0) == nv.Status.INVALID_ARG
+    assert call(E=300) == nv.Status.INVALID_ARG
+    assert call(K=96) == nv.Status.INVALID_ARG              # K % 32
+    assert call(K=320) == nv.Status.INVALID_ARG             # K % 256
+    assert call(off=0) == nv.Status.INVALID_ARG             # null offsets
+    assert call(ws=0) == nv.Status.INVALID_ARG              # no workspace
+    assert call(ws_bytes=need - 1) == nv.Status.INVALID_ARG  # too small
+    assert b"nvfp4_workspace_size" in lib.nvfp4_last_error()
+    assert call(A=24) == nv.Status.MISALIGNED
+    assert call(ws=4104) == nv.Status.MISALIGNED
+    assert call(M=0) == nv.Status.OK                        # nothing to do
+
+
+def test_prepare_scales_argument_errors_need_no_device():
+    lib = nv.load_library()
+    assert lib.nvfp4_prepare_scales(16, 16, 128, 96, None) == nv.Status.INVALID_ARG   # K % 64
+    assert lib.nvfp4_prepare_scales(0, 16, 128, 128, None) == nv.Status.INVALID_ARG
+    assert lib.nvfp4_prepare_scales(24, 16, 128, 128, None) == nv.Status.MISALIGNED
+    assert lib.nvfp4_prepare_scales(16, 16, 0, 128, None) == nv.Status.OK

@@ -74,6 +74,46 @@ def test_device_gA_equals_host_gA():
     assert torch.equal(ys[0].view(torch.int16), ys[1].view(torch.int16))
 
 
+def test_product_right_after_replanning_reads_the_new_schedule():
+    """The product is launched programmatically (it may start while the kernel before
+    it still runs); when that kernel is the schedule itself, the product must still
+    read the schedule only once it is complete.  Re-planning one buffer with new
+    offsets and launching the product straight after must give the new plan's result,
+    equal to the host-planned product's, every time."""
+    E, N, K = 3, 384, 512
+    plans = [[300, 5, 200], [10, 480, 15], [0, 0, 505], [256, 1, 248]]
+    M = sum(plans[0])
+    rng = np.random.default_rng(31)
+    A = wl.uniform_operand(rng, M, K)
+    Ws = [wl.uniform_operand(rng, N, K) for _ in range(E)]
+    Wc = _dev(np.stack([w.codes for w in Ws]))
+    gW = [0.5, 1.0, 2.0]
+    sw = nv.nvfp4_pack_scales_grouped(_dev(np.stack([w.scales for w in Ws]).reshape(E * N, -1)),
+                                      [e * N for e in range(E + 1)], K)
+    a_d, s_d = _dev(A.codes), _dev(A.scales)
+    offs, packed, expect = [], [], []
+    for counts in plans:
+        assert sum(counts) == M
+        off = [0] + list(np.cumsum(counts))
+        offs.append(torch.tensor(off, dtype=torch.int32, device="cuda"))
+        sa = nv.nvfp4_pack_scales_grouped(s_d, off, K)
+        pad = torch.zeros(nv.load_library().nvfp4_grouped_scale_layout_bytes_bound(M, E, K),
+                          dtype=torch.uint8, device="cuda")
+        pad[:sa.numel()] = sa
+        packed.append(pad)
+        expect.append(nv.gemm_nvfp4_w4a4_grouped_packed(a_d, sa, 1.25, Wc, sw, gW, off))
+    sched = nv.GroupedSchedule(offs[0], E, M, N, K, gW, gA=1.25)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    for rep in range(6):
+        for i in range(len(plans)):
+            sched.plan(offs[i], gW, gA=1.25)
+            sched.gemm(a_d, packed[i], Wc, sw, out=y)
+            torch.cuda.synchronize()
+            assert torch.equal(y.view(torch.int16), expect[i].view(torch.int16)), (rep, plans[i])
+    nv.nvfp4_check_device_error()
+
+
 def test_bad_device_offsets_are_reported_and_write_nothing():
     A, Wc, Ws, gW, off = _random_grouped([64, 64], 256, 256, 9)
     E, N, K, M = 2, 256, 256, 128
@@ -225,3 +265,30 @@ def test_fused_combine_reports_a_bad_destination_and_skips_it():
     assert bool((y[victim].float() == 3.0).all())                 # that token's row is not written
     others = [int(t) for t in L["src"].tolist() if int(t) != victim]
     assert not bool((y[others].float() == 3.0).all())
+
+
+@pytest.mark.parametrize("counts,N,K", COUNTS[:5])
+def test_plain_scale_entry_with_device_offsets(counts, N, K):
+    """gemm_nvfp4_w4a4_grouped: plain scales, device offsets and one caller workspace
+    (its size from nvfp4_workspace_size); equal to the host-planned packed product
+    bit for bit, and within tolerance of the oracle."""
+    A, Wc, Ws, gW, off = _random_grouped(counts, N, K, sum(counts) * 7 + N)
+    E, M = len(counts), int(off[-1])
+    need = nv.nvfp4_workspace_size(nv.Op.W4A4_GROUPED, M, N, K, E)
+    ws = torch.full((need,), 0xAB, dtype=torch.uint8, device="cuda")   # needs no zeroing
+    off_d = _dev(off.astype(np.int32))
+    y = nv.gemm_nvfp4_w4a4_grouped(_dev(A.codes), _dev(A.scales), 0.75, _dev(Wc), _dev(Ws), gW,
+                                   off_d, workspace=ws)
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    if M == 0:
+        return
+    sw = nv.nvfp4_pack_scales_grouped(_dev(Ws.reshape(E * N, K // 16)),
+                                      [e * N for e in range(E + 1)], K)
+    sa = nv.nvfp4_pack_scales_grouped(_dev(A.scales), list(off), K)
+    y_h = nv.gemm_nvfp4_w4a4_grouped_packed(_dev(A.codes), sa, 0.75, _dev(Wc), sw, list(gW),
+                                            list(off))
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y_h.view(torch.int16))
+    ref = oracle.gemm_grouped_w4a4(A.codes, A.scales, 0.75, Wc, Ws, gW, off, N, K)
+    check(bf16_to_f64(y), ref, f"grouped device offsets {counts}")
