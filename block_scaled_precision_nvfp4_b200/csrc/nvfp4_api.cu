@@ -1316,4 +1316,15 @@ nvfp4_status nvfp4_prepare_scales(const uint8_t* s_plain, uint8_t* s_mma, int ro
     return nvfp4_pack_scales(s_plain, rows, K, s_mma, stream);
 }
 
+#ifdef NVFP4_WAIT_TEST
+// Test-only build: sets the pipeline waits' time limit and the stall switch of
+// the single-SM W4A4 kernel on the current device.  Not in the product library.
+__attribute__((visibility("default"))) nvfp4_status nvfp4_test_set_wait(uint64_t limit_ns,
+                                                                        int stall) {
+    cudaError_t e = cudaMemcpyToSymbol(nvfp4::g_wait_limit_ns, &limit_ns, sizeof(limit_ns));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(nvfp4::g_wait_test_stall, &stall, sizeof(stall));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "setting the test wait variables");
+}
+#endif
+
 }  // extern "C"

@@ -18,6 +18,19 @@ __device__ int g_device_error = 0;
 // Time limit of every spin-wait, in nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+#ifdef NVFP4_WAIT_TEST
+// Test-only build (never the product library): the limit of the pipeline waits
+// and a switch that makes a kernel wait on a barrier nothing arms are device
+// variables the tests set, so that a bounded wait can be made to expire.
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+__device__ int g_wait_test_stall = 0;
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+    return *reinterpret_cast<volatile uint64_t*>(&g_wait_limit_ns);
+}
+#else
+__device__ __forceinline__ constexpr uint64_t wait_limit_ns() { return kWaitLimitNs; }
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -60,7 +73,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false (and
-// records `role` in the device error word) if the wait exceeds kWaitLimitNs
+// records `role` in the device error word) if the wait exceeds its time limit
 // or if another role of this CTA has already given up (*abort != 0).  Roles
 // that wait long and are not latency-critical pass `backoff_ns` so that their
 // polling does not take issue slots from the MMA and data-movement warps.
@@ -73,7 +86,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
         if (backoff_ns) __nanosleep(backoff_ns);
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > wait_limit_ns()) {
             *abort = 1;
             atomicOr(&g_device_error, 1 | (role << 8));
             return false;

@@ -17,19 +17,23 @@
 // an even group) or first chunk (odd group) is a shared all-zero tile, reached
 // through the smem descriptor's leading byte offset -- no zeros are copied.
 //
-// Roles (one persistent CTA per SM, 12 warps, 128 x 128 output tiles):
+// Roles (one persistent CTA per SM, 20 warps, 128 x 128 output tiles):
 //   warp 0      TMA producer: packed FP4 A/W K-blocks (256 codes, 128-byte
 //               swizzle) and their raw [rows][16 B] scale tiles.
 //   warp 1      TMEM owner, MMA issuer: one MMA per group into a 4-deep ring
 //               of 128-column FP32 partial buffers.
 //   warps 2-3   converters: FP4 -> E4M3 by the identity, into per-group
 //               [rows][16 B] operand tiles; scales -> FP32 (x 2^6).
-//   warps 4-11  scale-apply + epilogue: per group, partial TMEM -> registers,
-//               acc += P * (sA*64)(sW*64) with packed f32x2 FMAs; at the end of
-//               a tile, x alpha, BF16 RNE, store.
-// Every 16-group's 128 x 128 FP32 partial leaves TMEM to be scaled, so the
-// per-group chain (MMA, commit, partial read-out, FP32 apply) sets the pace, not
-// the FP8 tensor pipe.  Requires K % 256 == 0 (TMA of the scale tiles).
+//   warps 4-19  scale-apply + epilogue: warp w reads TMEM lane quarter w % 4
+//               (32 rows) and column slab (w - 4) / 4 (32 columns) of every
+//               partial, and adds P * (sA*64)(sW*64) with packed f32x2 FMAs into
+//               32 FP32 accumulators per thread; at the end of a tile, x alpha,
+//               BF16 RNE, store.
+// Every 16-group's 128 x 128 FP32 partial leaves TMEM to be scaled: two FP32
+// operations per output element per group (the scale product and the FMA), which
+// the FP32 pipe bounds, not the FP8 tensor pipe.  Sixteen apply warps keep four
+// TMEM reads and their arithmetic in flight per scheduler.  Requires
+// K % 256 == 0 (TMA of the scale tiles).
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -41,11 +45,14 @@ namespace via_fp8 {
 
 constexpr int BM = 128, BN = 128;
 constexpr int BK = 256;              // codes per raw K-block
-constexpr int RSTAGES = 3;           // raw K-block ring
+constexpr int RSTAGES = 4;           // raw K-block ring
 constexpr int NSLOTS = 4;            // converted group-pair ring
 constexpr int NPART = 4;             // TMEM partial buffers (128 columns each)
-constexpr int CONV_WARPS = 2, APPLY_WARPS = 8;
+constexpr int CONV_WARPS = 2, APPLY_WARPS = 16;
+constexpr int FIRST_APPLY = 2 + CONV_WARPS;       // a multiple of 4: warp % 4 = lane quarter
+constexpr int SLAB = BN / (APPLY_WARPS / 4);      // columns per apply warp (32)
 constexpr int NUM_THREADS = 32 * (2 + CONV_WARPS + APPLY_WARPS);
+static_assert(FIRST_APPLY % 4 == 0 && SLAB == 32, "apply warps: 4 per lane quarter, 32 columns each");
 constexpr int GROUP_M = 8;
 
 enum Role { ROLE_PRODUCER = 1, ROLE_MMA = 2, ROLE_CONV = 3, ROLE_APPLY = 4, ROLE_DRAIN = 5 };
@@ -97,6 +104,12 @@ __device__ __forceinline__ uint2 convert8(uint32_t w) {
     const uint32_t lo = e2m1_hi_to_e4m3((w << 4) & 0xF0F0F0F0u);  // k = 0, 2, 4, 6
     const uint32_t hi = e2m1_hi_to_e4m3(w & 0xF0F0F0F0u);         // k = 1, 3, 5, 7
     return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+}
+
+// Word i (0..3) of four held in registers, without indexing local memory.
+__device__ __forceinline__ uint32_t pick4(const uint32_t (&a)[4], int i) {
+    const uint32_t lo = (i & 1) ? a[1] : a[0], hi = (i & 1) ? a[3] : a[2];
+    return (i & 2) ? hi : lo;
 }
 
 // Non-negative E4M3 scale byte -> its value times 2^6, as FP32 (exact).
@@ -256,7 +269,6 @@ via_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 for (int h = 0; h < 8; ++h, ++pc) {
                     const int sl = pc % NSLOTS;
                     if (!warp_wait(&sm.slot_empty[sl], ((pc / NSLOTS) & 1) ^ 1, abort, ROLE_CONV)) { ok = false; break; }
-                    const int g0 = 2 * h, g1 = 2 * h + 1;
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr) {
                         const int row = ctid + 64 * rr;
@@ -270,10 +282,13 @@ via_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         *reinterpret_cast<uint4*>(sm.a8[sl][1] + row * 16) = make_uint4(a2.x, a2.y, a3.x, a3.y);
                         *reinterpret_cast<uint4*>(sm.b8[sl][0] + row * 16) = make_uint4(b0.x, b0.y, b1.x, b1.y);
                         *reinterpret_cast<uint4*>(sm.b8[sl][1] + row * 16) = make_uint4(b2.x, b2.y, b3.x, b3.y);
-                        sm.sa_f[sl][0][row] = scale_x64((saw[rr][g0 >> 2] >> (8 * (g0 & 3))) & 0xFFu);
-                        sm.sa_f[sl][1][row] = scale_x64((saw[rr][g1 >> 2] >> (8 * (g1 & 3))) & 0xFFu);
-                        sm.sw_f[sl][0][row] = scale_x64((sbw[rr][g0 >> 2] >> (8 * (g0 & 3))) & 0xFFu);
-                        sm.sw_f[sl][1][row] = scale_x64((sbw[rr][g1 >> 2] >> (8 * (g1 & 3))) & 0xFFu);
+                        // scale bytes g0 = 2h and g1 = 2h + 1: bytes 2(h&1), 2(h&1)+1 of word h/2
+                        const uint32_t wa = pick4(saw[rr], h >> 1) >> (16 * (h & 1));
+                        const uint32_t wb = pick4(sbw[rr], h >> 1) >> (16 * (h & 1));
+                        sm.sa_f[sl][0][row] = scale_x64(wa & 0xFFu);
+                        sm.sa_f[sl][1][row] = scale_x64((wa >> 8) & 0xFFu);
+                        sm.sw_f[sl][0][row] = scale_x64(wb & 0xFFu);
+                        sm.sw_f[sl][1][row] = scale_x64((wb >> 8) & 0xFFu);
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -286,17 +301,17 @@ via_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ scale-apply + epilogue
-        const int q = warp & 3;                       // TMEM lane quarter
-        const int half = (warp - 2 - CONV_WARPS) >> 2;  // column half
-        const int trow = 32 * q + lane;               // row within the tile
+        const int q = warp & 3;                    // TMEM lane quarter
+        const int slab = (warp - FIRST_APPLY) >> 2;  // 32-column slab of the tile
+        const int trow = 32 * q + lane;            // row within the tile
         const bool vec_ok = (N % 8) == 0;
         int pc = 0, gc = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
             int mb, nb;
             tile_coords(tile, num_m, num_n, mb, nb);
-            uint64_t acc[32];
+            uint64_t acc[SLAB / 2];  // FP32 pairs
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] = 0ull;
+            for (int j = 0; j < SLAB / 2; ++j) acc[j] = 0ull;
             bool ok = true;
             for (int pair = 0; pair < num_kb * 8 && ok; ++pair, ++pc) {
                 const int sl = pc % NSLOTS;
@@ -306,53 +321,54 @@ via_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     const int p = gc % NPART;
                     if (!warp_wait(&sm.part_full[p], (gc / NPART) & 1, abort, ROLE_APPLY)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + p * 128 + half * 64;
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + p * 128 + slab * SLAB, v);
+                    tmem_ld_wait();
+                    reg_fence(v);
+                    // the partial is in registers: hand its columns back to the MMA
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.part_empty[p]);
+                    // acc += P * ((sA*64) * (sW*64)): the scale product has at most 8
+                    // significant bits and P*S at most 22, so both are exact and the FMA
+                    // rounds once, into the accumulator (packed f32x2 lanes)
                     const float sa = sm.sa_f[sl][gi][trow];
                     const uint64_t sa2 = pack2(__float_as_uint(sa), __float_as_uint(sa));
-                    const uint64_t* sw2 = reinterpret_cast<const uint64_t*>(&sm.sw_f[sl][gi][half * 64]);
+                    const float4* sw4 = reinterpret_cast<const float4*>(&sm.sw_f[sl][gi][slab * SLAB]);
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(ta + 32 * c, v);
-                        tmem_ld_wait();
-                        reg_fence(v);
-                        if (c == 1) {  // the whole partial is in registers: release it
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&sm.part_empty[p]);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            acc[16 * c + j] = fma2(pack2(v[2 * j], v[2 * j + 1]),
-                                                   mul2(sa2, sw2[16 * c + j]), acc[16 * c + j]);
+                    for (int i = 0; i < SLAB / 4; ++i) {
+                        const float4 w4 = sw4[i];
+                        const uint64_t s01 = mul2(sa2, pack2(__float_as_uint(w4.x), __float_as_uint(w4.y)));
+                        const uint64_t s23 = mul2(sa2, pack2(__float_as_uint(w4.z), __float_as_uint(w4.w)));
+                        acc[2 * i] = fma2(pack2(v[4 * i], v[4 * i + 1]), s01, acc[2 * i]);
+                        acc[2 * i + 1] = fma2(pack2(v[4 * i + 2], v[4 * i + 3]), s23, acc[2 * i + 1]);
                     }
                 }
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(&sm.slot_empty[sl]);
             }
             if (!ok) break;
-            // epilogue: x alpha, BF16 RNE, store this thread's 64 columns
+            // epilogue: x alpha, BF16 RNE, store this thread's 32 columns
             const int row = mb * BM + trow;
-            const int col0 = nb * BN + half * 64;
+            const int col0 = nb * BN + slab * SLAB;
             if (row < M) {
-                uint32_t packed[32];
+                uint32_t packed[SLAB / 2];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float lo = __uint_as_float((uint32_t)acc[j]) * alpha;
-                    const float hi = __uint_as_float((uint32_t)(acc[j] >> 32)) * alpha;
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
+                for (int j = 0; j < SLAB / 2; ++j) {
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float((uint32_t)acc[j]), alpha),
+                                                              __fmul_rn(__uint_as_float((uint32_t)(acc[j] >> 32)), alpha));
                     packed[j] = *reinterpret_cast<uint32_t*>(&h2);
                 }
                 __nv_bfloat16* yrow = Y + (size_t)row * N;
-                if (vec_ok && col0 + 64 <= N) {
+                if (vec_ok && col0 + SLAB <= N) {
                     uint4* dst = reinterpret_cast<uint4*>(yrow + col0);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
+                    for (int j = 0; j < SLAB / 8; ++j)
                         dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
                 } else {
                     uint16_t* y16 = reinterpret_cast<uint16_t*>(yrow);
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
+                    for (int j = 0; j < SLAB; ++j)
                         if (col0 + j < N) y16[col0 + j] = (uint16_t)(packed[j >> 1] >> (16 * (j & 1)));
                 }
             }

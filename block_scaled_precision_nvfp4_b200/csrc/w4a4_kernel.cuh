@@ -55,6 +55,9 @@ struct Smem {
     uint64_t acc_full;
     uint64_t acc_empty;
     uint64_t drain;
+#ifdef NVFP4_WAIT_TEST
+    uint64_t never;  // test-only: a barrier nothing arrives on
+#endif
     uint32_t tmem_base;
     int abort;
 };
@@ -150,6 +153,9 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.acc_empty, NUM_EPI_WARPS);
         mbar_init(&sm.drain, 1);
+#ifdef NVFP4_WAIT_TEST
+        mbar_init(&sm.never, 1);
+#endif
         sm.abort = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&tmA);
@@ -211,6 +217,11 @@ w4a4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         const uint32_t idesc = idesc_mxf4nvf4(BM, BN);
         int it = 0, tc = 0;
         bool ok = true;
+#ifdef NVFP4_WAIT_TEST
+        // test-only: wait on a barrier nothing arms, so that this bounded wait
+        // expires and every role of the CTA takes its abort path
+        if (g_wait_test_stall && !warp_wait(&sm.never, 0, abort, ROLE_MMA)) ok = false;
+#endif
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
             if (!warp_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
             tc_fence_after();

@@ -42,3 +42,42 @@ def packed_reference(s, K):
     pad[:rows] = s
     v = pad.reshape(rb_n, 4, 32, K // 64, 4)          # [rb][j][i][ks][t]
     return np.ascontiguousarray(v.transpose(0, 3, 2, 1, 4)).ravel()  # [rb][ks][i][j][t]
+
+
+class Accum:
+    """check() for a result compared in pieces: the same tolerances, on the whole.
+
+    add(y, ref) takes one piece; finish(count) asserts that exactly `count` elements
+    were compared and that the relative Frobenius error and max |err| / max |ref| of
+    the whole result are within REL_FRO_TOL and MAX_ABS_REL_TOL."""
+
+    def __init__(self, what=""):
+        self.what = what
+        self.n = 0
+        self.err2 = 0.0
+        self.ref2 = 0.0
+        self.max_err = 0.0
+        self.max_ref = 0.0
+
+    def add(self, y, ref):
+        y = np.asarray(y, dtype=np.float64)
+        ref = np.asarray(ref, dtype=np.float64)
+        assert y.shape == ref.shape, f"{self.what}: shape {y.shape} != {ref.shape}"
+        assert np.all(np.isfinite(ref)), f"{self.what}: non-finite reference"
+        assert np.all(np.isfinite(y)), f"{self.what}: non-finite result"
+        d = y - ref
+        self.n += y.size
+        self.err2 += float(np.sum(d * d))
+        self.ref2 += float(np.sum(ref * ref))
+        if y.size:
+            self.max_err = max(self.max_err, float(np.max(np.abs(d))))
+            self.max_ref = max(self.max_ref, float(np.max(np.abs(ref))))
+
+    def finish(self, count):
+        assert self.n == count, f"{self.what}: compared {self.n} elements, expected {count}"
+        assert self.n > 0 and self.ref2 > 0, f"{self.what}: empty or all-zero reference"
+        rel = np.sqrt(self.err2 / self.ref2)
+        mx = self.max_err / self.max_ref
+        assert rel <= REL_FRO_TOL, f"{self.what}: relative Frobenius error {rel:.3e} > {REL_FRO_TOL}"
+        assert mx <= MAX_ABS_REL_TOL, f"{self.what}: max |err|/max|ref| {mx:.3e} > {MAX_ABS_REL_TOL}"
+        return rel, mx
