@@ -250,24 +250,19 @@ nvfp4_status set_smem(Kern k, size_t bytes, const DevInfo& info, const char* nam
     return NVFP4_OK;
 }
 
-using W4a16Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                           const uint16_t*, const uint8_t*, __nv_bfloat16*, int, int, int, float, int);
-template <int NB>
-W4a16Kern w4a16_inst(bool sf_tma) {
-    return sf_tma ? nvfp4::w4a16::w4a16_kernel<NB, true> : nvfp4::w4a16::w4a16_kernel<NB, false>;
-}
-// the instantiation for `nb` row blocks per CTA (1..MAX_NB)
-W4a16Kern w4a16_kernel_for(int nb, bool sf_tma) {
-    static_assert(nvfp4::w4a16::MAX_NB == 8, "one instantiation per row-block count");
+using W4a16LdgKern = void (*)(const uint16_t*, const uint8_t*, const uint8_t*, __nv_bfloat16*, int,
+                              int, int, float, int);
+// the register-load instantiation for `nb` row blocks per CTA (1..LDG_MAX_NB)
+W4a16LdgKern w4a16_ldg_kernel_for(int nb) {
+    namespace k16 = nvfp4::w4a16;
+    static_assert(k16::LDG_MAX_NB == 6, "one instantiation per row-block count");
     switch (nb) {
-        case 1: return w4a16_inst<1>(sf_tma);
-        case 2: return w4a16_inst<2>(sf_tma);
-        case 3: return w4a16_inst<3>(sf_tma);
-        case 4: return w4a16_inst<4>(sf_tma);
-        case 5: return w4a16_inst<5>(sf_tma);
-        case 6: return w4a16_inst<6>(sf_tma);
-        case 7: return w4a16_inst<7>(sf_tma);
-        default: return w4a16_inst<8>(sf_tma);
+        case 1: return k16::w4a16_ldg_kernel<1>;
+        case 2: return k16::w4a16_ldg_kernel<2>;
+        case 3: return k16::w4a16_ldg_kernel<3>;
+        case 4: return k16::w4a16_ldg_kernel<4>;
+        case 5: return k16::w4a16_ldg_kernel<5>;
+        default: return k16::w4a16_ldg_kernel<6>;
     }
 }
 
@@ -846,47 +841,24 @@ nvfp4_status gemm_w4a16(const void* A, const uint8_t* W, const uint8_t* sW, floa
     if (M == 0 || N == 0) return ok();
 
     // one wave: blocks of 8 weight rows spread evenly over the SMs, at most
-    // MAX_NB per CTA (more CTAs than SMs only for very tall W)
+    // LDG_MAX_NB per CTA (more CTAs than SMs only for very tall W)
     const int nrb = (N + k16::ROWS - 1) / k16::ROWS;
     int grid = nrb < info.num_sms ? nrb : info.num_sms;
     int nb = (nrb + grid - 1) / grid;
-    if (nb > k16::MAX_NB) {
-        nb = k16::MAX_NB;
+    if (nb > k16::LDG_MAX_NB) {
+        nb = k16::LDG_MAX_NB;
         grid = (nrb + nb - 1) / nb;
     }
-    // codes by TMA always (K % 32 == 0 keeps the row pitch a multiple of 16 bytes);
-    // scales by TMA when their row pitch K/16 is a multiple of 16 bytes too
-    const bool sf_tma = K % 256 == 0;
-    nvfp4_status st;
-    // boxes of all of a CTA's rows: CTAs own nb or nb - 1 blocks of 8 rows
-    CUtensorMap tmW, tmW1, tmS, tmS1;
-    memset(&tmW1, 0, sizeof(tmW1));
-    memset(&tmS, 0, sizeof(tmS));
-    memset(&tmS1, 0, sizeof(tmS1));
-    const uint32_t rows = (uint32_t)nb * k16::ROWS;
-    if ((st = make_map_u8(&tmW, W, (uint64_t)K / 2, (uint64_t)N, 128, rows)) != NVFP4_OK) return st;
-    if (nb > 1 && (st = make_map_u8(&tmW1, W, (uint64_t)K / 2, (uint64_t)N, 128, rows - k16::ROWS)) != NVFP4_OK)
-        return st;
-    if (sf_tma) {
-        if ((st = make_map_u8(&tmS, sW, (uint64_t)K / 16, (uint64_t)N, 64, rows,
-                              CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
-            return st;
-        if (nb > 1 && (st = make_map_u8(&tmS1, sW, (uint64_t)K / 16, (uint64_t)N, 64, rows - k16::ROWS,
-                                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4_OK)
-            return st;
-    }
-    W4a16Kern kern = w4a16_kernel_for(nb, sf_tma);
-    const size_t smem = k16::smem_bytes(nb);
-    if ((st = set_smem(kern, smem, info, "w4a16_kernel")) != NVFP4_OK) return st;
+    W4a16LdgKern kern = w4a16_ldg_kernel_for(nb);
     const float out_scale = 128.0f * gW;  // undoes the 2^-7 carried by the widened weights
     for (int m0 = 0; m0 < M; m0 += k16::TOK) {
         const int mc = M - m0 < k16::TOK ? M - m0 : k16::TOK;
         const uint16_t* a = static_cast<const uint16_t*>(A) + (size_t)m0 * K;
         __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y) + (size_t)m0 * N;
-        kern<<<grid, k16::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
-            tmW, tmW1, tmS, tmS1, a, sW, y, mc, N, K, out_scale, nrb);
+        kern<<<grid, k16::LDG_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+            a, W, sW, y, mc, N, K, out_scale, nrb);
         cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "launching w4a16_kernel");
+        if (e != cudaSuccess) return cuda_fail(e, "launching w4a16_ldg_kernel");
     }
     return ok();
 }
