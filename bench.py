@@ -298,8 +298,90 @@ KERNEL_SOURCES = {
     "grouped": ["grouped_pair_kernel.cuh", "w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh"],
     "moe": ["grouped_pair_kernel.cuh", "w4a4_pair_kernel.cuh", "w4a4_kernel.cuh", "ptx.cuh",
             "moe_kernel.cuh", "quantize_kernel.cuh"],
-    "quantize": ["quantize_kernel.cuh"],
+    "quantize": ["quantize_kernel.cuh", "ptx.cuh"],
 }
+
+
+# The per-update FP32 work of the exact paths' scale-apply, measured on the device
+# itself: a kernel of independent chains, each step one scale product and one FMA
+# into an accumulator (no loop-invariant operand a compiler could hoist), written
+# once with scalar FP32 instructions and once with packed f32x2 ones.  The larger
+# rate is the roofline's peak.
+APPLY_PEAK_SRC = r"""
+#include <cstdio>
+#include <cstdint>
+#include <cuda_runtime.h>
+template <int PACKED>
+__global__ void __launch_bounds__(256, 1) apply_peak(float* out, int iters, long long* cyc) {
+    uint64_t a[16], sc[16];
+    const uint64_t p = 0x3f8000013f800001ull;
+    const uint64_t c = 0x3f8000003f800000ull ^ (uint64_t)(threadIdx.x & 1);
+    for (int j = 0; j < 16; ++j) { a[j] = (uint64_t)(threadIdx.x + j) * 0x0000000100000001ull; sc[j] = 0x3f0000003f000000ull + j; }
+    const long long t0 = clock64();
+    for (int i = 0; i < iters; ++i) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (PACKED) {
+                asm volatile("mul.rn.f32x2 %0, %0, %1;" : "+l"(sc[j]) : "l"(c));
+                asm volatile("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a[j]) : "l"(p), "l"(sc[j]));
+            } else {
+                float s0 = __uint_as_float((uint32_t)sc[j]), s1 = __uint_as_float((uint32_t)(sc[j] >> 32));
+                float x0 = __uint_as_float((uint32_t)a[j]), x1 = __uint_as_float((uint32_t)(a[j] >> 32));
+                asm volatile("mul.rn.f32 %0, %0, %1;" : "+f"(s0) : "f"(__uint_as_float((uint32_t)c)));
+                asm volatile("mul.rn.f32 %0, %0, %1;" : "+f"(s1) : "f"(__uint_as_float((uint32_t)c)));
+                asm volatile("fma.rn.f32 %0, %1, %2, %0;" : "+f"(x0) : "f"(1.0000001f), "f"(s0));
+                asm volatile("fma.rn.f32 %0, %1, %2, %0;" : "+f"(x1) : "f"(1.0000001f), "f"(s1));
+                sc[j] = (uint64_t)__float_as_uint(s0) | ((uint64_t)__float_as_uint(s1) << 32);
+                a[j] = (uint64_t)__float_as_uint(x0) | ((uint64_t)__float_as_uint(x1) << 32);
+            }
+        }
+    }
+    const long long t1 = clock64();
+    uint64_t x = 0;
+    for (int j = 0; j < 16; ++j) x ^= a[j] ^ sc[j];
+    out[blockIdx.x * blockDim.x + threadIdx.x] = (float)(x & 0xffff);
+    if (threadIdx.x == 0) cyc[blockIdx.x] = t1 - t0;
+}
+template <int PACKED> double rate(int sms, float* out, long long* cyc) {
+    const int iters = 4096, threads = 256;
+    apply_peak<PACKED><<<sms, threads>>>(out, 2, cyc);
+    apply_peak<PACKED><<<sms, threads>>>(out, iters, cyc);
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1.0;
+    long long h[1024];
+    cudaMemcpy(h, cyc, sizeof(long long) * sms, cudaMemcpyDeviceToHost);
+    double mx = 0;
+    for (int b = 0; b < sms; ++b) mx = h[b] > mx ? (double)h[b] : mx;
+    return 32.0 * threads * iters / mx;  // updates per clock per SM (two per j per thread)
+}
+int main() {
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, 0);
+    float* out; long long* cyc;
+    if (cudaMalloc(&out, sizeof(float) * sms * 256) != cudaSuccess || cudaMalloc(&cyc, 8 * 1024) != cudaSuccess) return 1;
+    printf("scalar %.2f\npacked %.2f\n", rate<0>(sms, out, cyc), rate<1>(sms, out, cyc));
+    return 0;
+}
+"""
+
+
+def measure_apply_peak():
+    """Scale-apply updates per clock per SM (scalar, packed), from APPLY_PEAK_SRC compiled
+    with nvcc into _build/ (cached by source hash) and run on the current device."""
+    import subprocess
+    h = hashlib.sha256(APPLY_PEAK_SRC.encode()).hexdigest()[:16]
+    d = os.path.join(ROOT, "_build")
+    os.makedirs(d, exist_ok=True)
+    exe = os.path.join(d, f"apply_peak_{h}")
+    if not os.path.exists(exe):
+        src = exe + ".cu"
+        with open(src, "w") as f:
+            f.write(APPLY_PEAK_SRC)
+        nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+        subprocess.check_call([nvcc if os.path.exists(nvcc) else "nvcc", "-gencode",
+                               "arch=compute_100a,code=sm_100a", "-O3", "-o", exe, src])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120, check=True).stdout
+    vals = dict(line.split() for line in out.strip().splitlines())
+    return float(vals["scalar"]), float(vals["packed"])
 
 
 def kernel_source_hash(path):
@@ -313,7 +395,9 @@ def kernel_source_hash(path):
 
 def profiled_traffic(workload_name, path):
     """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
-    fn = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.txt")
+    fn = os.path.join(ROOT, "profiles", f"traffic_{path}_{workload_name}.txt")
+    if not os.path.exists(fn):
+        fn = os.path.join(ROOT, "profiles", f"traffic_{workload_name}.txt")
     try:
         kv = {}
         with open(fn) as f:
@@ -671,7 +755,7 @@ def run_ours(args):
                  "permute_gbs": 2 * M * (K // 2 + K // 16) / (med["permute"] * 1e-6) / 1e9}
     kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel", "w4a8": "w4a8_kernel",
                    "moe": "grouped_pair_kernel",
-                   "w4a16": "w4a16_kernel", "grouped": "grouped_pair_kernel",
+                   "w4a16": "w4a16_ldg_kernel", "grouped": "grouped_pair_kernel",
                    "quantize": "quantize_bf16_kernel (+ amax_bf16_kernel)"}[path]
     if spec["bound"] == "tensor_fp8":
         # the W4A8 kernel runs three E4M3 x E5M2 MMAs per K step (one per signed digit of
@@ -717,18 +801,25 @@ def run_ours(args):
                                                        else "weight codes")
                                + " after the same flush; GB/s counts read + write")}
     else:
-        # each (row, column, group) update is FP32 work on 128 FP32 lanes per SM: two
-        # operations on the W4A4 exact path (the scale product and the FMA into the
-        # accumulator), one on the W4A8 path (the weights' scale only: one FMA)
-        ops = 1 if path == "w4a8" else 2
+        # The W4A4 exact path does two FP32 operations per (row, column, group) update:
+        # the scale product and the FMA into the accumulator; its peak is the measured
+        # rate of that pair on this device, scalar or packed, whichever is higher, at the
+        # maximum SM clock.  The W4A8 path's FP32 work is one FMA per update; its peak is
+        # SMs x 128 FP32 lanes x max clock.
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         clk_mhz = clk.summary().get("sm_max_mhz") or 1965
-        peak_upd = sms * (128 // ops) * clk_mhz * 1e6 / 1e12  # T updates / s
+        if path == "w4a8":
+            per_clk, note = 128.0, "one FMA per update: SMs x 128 FP32 lanes x max clock"
+        else:
+            scalar, packed = measure_apply_peak()
+            per_clk = max(scalar, packed)
+            note = (f"measured scale product + FMA per update on this device: {scalar:.1f} "
+                    f"(scalar FP32) / {packed:.1f} (packed f32x2) updates per clock per SM; "
+                    f"peak = SMs x the larger x max clock")
+        peak_upd = sms * per_clk * clk_mhz * 1e6 / 1e12  # T updates / s
         achieved = (M * N * K / 16) / kern_s / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": peak_upd,
-                "unit": "Tupdate/s", "frac": achieved / peak_upd,
-                "peak_note": (f"per-16 FP32 scale-apply updates, {ops} FP32 op(s) each; derived: "
-                              f"SMs x 128 FP32 lanes / {ops} x max clock")}
+                "unit": "Tupdate/s", "frac": achieved / peak_upd, "peak_note": note}
     roof.update({"traffic": profiled_traffic(wl_.name, path), "kernel": kernel_name,
                  "kernel_ms": kern_s * 1e3})
     roof.update(extra)

@@ -483,9 +483,21 @@ nvfp4_status nvfp4_quantize_bf16(const void* X, int rows, int K, uint8_t* codes,
     const dim3 grid((unsigned)(rows > 0 ? (rows + q::TILE_ROWS - 1) / q::TILE_ROWS : 1),
                     (unsigned)((K + q::TILE_COLS - 1) / q::TILE_COLS));
     if (grid.y > 65535) return fail(NVFP4_ERR_INVALID_ARG, "K too large (got %d)", K);
-    q::quantize_bf16_kernel<<<grid, q::THREADS, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(X), rows, K, amax, codes, scales, scales_packed, g_out);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launching quantize_bf16_kernel");
+    // launched programmatically: its CTAs may start (and read X) while the amax kernel
+    // finishes; they read the maximum only after griddepcontrol.wait
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(q::THREADS);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, q::quantize_bf16_kernel, static_cast<const __nv_bfloat16*>(X), rows,
+                           K, static_cast<const unsigned*>(amax), codes, scales, scales_packed, g_out);
+    if (e != cudaSuccess) return cuda_fail(e, "launching quantize_bf16_kernel");
     return ok();
 }
 

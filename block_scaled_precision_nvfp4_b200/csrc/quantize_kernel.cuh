@@ -19,6 +19,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace nvfp4 {
 namespace quant {
 
@@ -32,6 +34,9 @@ constexpr int QB = 4;            // row segments of a warp in flight at once
 __global__ void __launch_bounds__(AMAX_THREADS)
 amax_bf16_kernel(const uint4* __restrict__ x, size_t n16, const uint16_t* __restrict__ tail,
                  int ntail, unsigned* amax_bits) {
+    // the quantiser launched after this kernel may start now: it reads X ahead and
+    // waits for this grid (griddepcontrol.wait) before it reads the maximum
+    grid_dependents_launch();
     unsigned m = 0;
     for (size_t i = blockIdx.x * (size_t)AMAX_THREADS + threadIdx.x; i < n16;
          i += (size_t)gridDim.x * AMAX_THREADS) {
@@ -110,23 +115,30 @@ quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
     __shared__ uint32_t sc[TILE_ROWS][TILE_COLS / 64 + 1];  // [row][K=64 step] four scale bytes
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blockIdx.x * TILE_ROWS, c0 = blockIdx.y * TILE_COLS;
-    const float g = global_scale(*amax_bits);
-    const float d6 = __fmul_rn(6.0f, g);
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
     const int col = c0 + 8 * lane;
     const bool col_ok = col < K;  // K % 16 == 0: a lane's 8 columns are all in or all out
 
     // this warp's 16 row segments, QB at a time in flight before any is used
     constexpr int RPW = TILE_ROWS / 8;  // rows per warp
-#pragma unroll 1
-    for (int i0 = 0; i0 < RPW; i0 += QB) {
-        uint4 vin[QB];
+    uint4 vin[QB];
+    auto load_rows = [&](int i0) {
 #pragma unroll
         for (int i = 0; i < QB; ++i) {
             const int row = r0 + warp * RPW + i0 + i;
             vin[i] = make_uint4(0u, 0u, 0u, 0u);
             if (col_ok && row < rows) vin[i] = __ldcs(reinterpret_cast<const uint4*>(X + (size_t)row * K + col));
         }
+    };
+    // The first rows are read while the amax kernel before this one may still run
+    // (programmatic launch); the maximum is read only after that grid has completed.
+    load_rows(0);
+    grid_dependency_wait();
+    const float g = global_scale(__ldcg(amax_bits));
+    const float d6 = __fmul_rn(6.0f, g);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
+#pragma unroll 1
+    for (int i0 = 0; i0 < RPW; i0 += QB) {
+        if (i0 > 0) load_rows(i0);
 #pragma unroll
     for (int i = 0; i < QB; ++i) {
         const int rl = warp * RPW + i0 + i;
