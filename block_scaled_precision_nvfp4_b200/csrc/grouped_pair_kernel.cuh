@@ -349,7 +349,7 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
                 int dest = tl.m0 + rbase + lane;
                 float f = alpha;
                 if (row_dest) row_target(row_dest, row_w, dest_rows, rbase + lane < tl.rows, alpha, dest, f);
-                if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI, 256)) break;
+                if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI)) break;
                 tc_fence_after();
                 uint32_t packed[COLS / 2];
 #pragma unroll
@@ -388,7 +388,7 @@ grouped_pair_kernel(const __grid_constant__ CUtensorMap tmA,    // A codes, box 
                     row_target(row_dest, row_w, dest_rows, tok0 + lane < tl.rows, alpha, d0, f0);
                     row_target(row_dest, row_w, dest_rows, tok0 + 32 + lane < tl.rows, alpha, d1, f1);
                 }
-                if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI, 256)) break;
+                if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI)) break;
                 tc_fence_after();
                 uint32_t tok2[32];  // BF16 pairs of consecutive tokens
 #pragma unroll

@@ -183,62 +183,74 @@ via_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int it = 0;
-            for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
-                int mb, nb;
-                tile_coords(tile, num_m, num_n, mb, nb);
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int r = it % RSTAGES;
-                    if (!mbar_wait(&sm.raw_empty[r], ((it / RSTAGES) & 1) ^ 1, abort, ROLE_PRODUCER))
-                        goto producer_done;
+        // The whole warp walks the loop (converged); one elected lane issues.
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            int mb, nb;
+            tile_coords(tile, num_m, num_n, mb, nb);
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int r = it % RSTAGES;
+                if (!warp_wait(&sm.raw_empty[r], ((it / RSTAGES) & 1) ^ 1, abort, ROLE_PRODUCER)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
                     mbar_arrive_expect_tx(&sm.raw_full[r], RAW_BYTES);
                     tma_load_2d(sm.raw_a[r], &tmA, &sm.raw_full[r], kb * 128, mb * BM);
                     tma_load_2d(sm.raw_b[r], &tmB, &sm.raw_full[r], kb * 128, nb * BN);
                     tma_load_2d(sm.raw_sa[r], &tmSA, &sm.raw_full[r], kb * 16, mb * BM);
                     tma_load_2d(sm.raw_sb[r], &tmSB, &sm.raw_full[r], kb * 16, nb * BN);
                 }
+                __syncwarp();
             }
-        producer_done:
-            if (*abort) {
-                for (int j = max(0, it - RSTAGES); j < it; ++j) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(&sm.raw_full[j % RSTAGES], (j / RSTAGES) & 1) &&
-                           globaltimer_ns() - t0 < kWaitLimitNs) {
-                    }
+        }
+        if (!ok && lane == 0) {
+            // every copy this warp started lands before the CTA can exit
+            for (int j = max(0, it - RSTAGES); j < it; ++j) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&sm.raw_full[j % RSTAGES], (j / RSTAGES) & 1) &&
+                       globaltimer_ns() - t0 < kWaitLimitNs) {
                 }
             }
         }
+        __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_f8f6f4_e4m3(BM, BN);
-            const uint32_t zlo = smem_u32(sm.zlo), zhi = smem_u32(sm.zhi);
-            int pc = 0, gc = 0;
-            for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-                bool ok = true;
-                for (int pair = 0; pair < num_kb * 8 && ok; ++pair, ++pc) {
-                    const int sl = pc % NSLOTS;
-                    if (!mbar_wait(&sm.slot_full[sl], (pc / NSLOTS) & 1, abort, ROLE_MMA)) { ok = false; break; }
-                    const uint32_t a_even = smem_u32(sm.a8[sl][0]), a_odd = smem_u32(sm.a8[sl][1]);
-                    const uint32_t b0 = smem_u32(sm.b8[sl][0]), b1 = smem_u32(sm.b8[sl][1]);
-                    // B: the K = 32 slice holding both groups of the pair
-                    const uint64_t bdesc = smem_desc(b0, b1 - b0, 128, 0);
+        // The whole warp walks the loop (converged, as tcgen05 issue wants it); the
+        // same elected lane issues every MMA and every commit that tracks them.
+        const uint32_t idesc = idesc_f8f6f4_e4m3(BM, BN);
+        const uint32_t zlo = smem_u32(sm.zlo), zhi = smem_u32(sm.zhi);
+        int pc = 0, gc = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            for (int pair = 0; pair < num_kb * 8 && ok; ++pair, ++pc) {
+                const int sl = pc % NSLOTS;
+                if (!warp_wait(&sm.slot_full[sl], (pc / NSLOTS) & 1, abort, ROLE_MMA)) { ok = false; break; }
+                const uint32_t a_even = smem_u32(sm.a8[sl][0]), a_odd = smem_u32(sm.a8[sl][1]);
+                const uint32_t b0 = smem_u32(sm.b8[sl][0]), b1 = smem_u32(sm.b8[sl][1]);
+                // B: the K = 32 slice holding both groups of the pair
+                const uint64_t bdesc = smem_desc(b0, b1 - b0, 128, 0);
 #pragma unroll
-                    for (int gi = 0; gi < 2; ++gi, ++gc) {
-                        const int p = gc % NPART;
-                        if (!mbar_wait(&sm.part_empty[p], ((gc / NPART) & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
-                        tc_fence_after();
+                for (int gi = 0; gi < 2; ++gi, ++gc) {
+                    const int p = gc % NPART;
+                    if (!warp_wait(&sm.part_empty[p], ((gc / NPART) & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
+                    tc_fence_after();
+                    if (elect_one()) {
                         // A: this group's 16 bytes in one K chunk, the other chunk all zero
                         const uint64_t adesc = gi == 0 ? smem_desc(a_even, zhi - a_even, 128, 0)
                                                        : smem_desc(zlo, a_odd - zlo, 128, 0);
                         mma_f8f6f4(tmem + p * 128, adesc, bdesc, idesc, 0u);
                         mma_commit(&sm.part_full[p]);
                     }
-                    if (ok) mma_commit(&sm.slot_empty[sl]);
+                    __syncwarp();
                 }
-                if (!ok) break;
+                if (ok && elect_one()) mma_commit(&sm.slot_empty[sl]);
+                __syncwarp();
             }
+        }
+        // every MMA issued completes before TMEM is freed
+        if (elect_one()) {
             mma_commit(&sm.drain);
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&sm.drain, 0)) {
@@ -248,6 +260,7 @@ via_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
             }
         }
+        __syncwarp();
     } else if (warp < 2 + CONV_WARPS) {
         // ------------------------------------------------------------ converters
         const int ctid = threadIdx.x - 64;  // 0..63: rows ctid and ctid + 64 of A and of W

@@ -66,7 +66,7 @@ constexpr int STAGES = 5;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int NUM_THREADS = 32 * (2 + NUM_EPI_WARPS);
 constexpr int FIRST_EPI_WARP = 2;
-constexpr int GROUP_M = 8;
+constexpr int GROUP_M = 16;
 
 struct Smem {
     alignas(1024) uint8_t a[STAGES][BM * BKB];
@@ -442,7 +442,7 @@ w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmA,   // A codes, box 128 
         for (int j = 0; segment_of(j, cid, nclusters, tiles, dp_tiles, num_kb, sg); ++j, ++tc) {
             int mb, nb;
             tile_coords(sg.tile, num_m, num_n, mb, nb);
-            if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI, 256)) break;
+            if (!warp_wait(&sm.acc_full, tc & 1, abort, ROLE_EPI)) break;
             tc_fence_after();
             // the whole accumulator block behind one wait, then TMEM goes back to the MMA
             uint32_t r[CHUNKS][32];

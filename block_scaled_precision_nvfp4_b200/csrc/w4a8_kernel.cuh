@@ -279,25 +279,27 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_f8f6f4(BW, BT, /*A E5M2*/ 1u, /*B E4M3*/ 0u);
-            // descriptor of stage 0's first K slice; stage a and slice hh add their offsets
-            // (in 16-byte units) to the start-address field
-            const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(sm.act[0]));
-            int ait = 0, it = 0, tc = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
-                // the epilogue has read the previous tile's accumulator
-                if (!mbar_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
-                tc_fence_after();
-                for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
-                    for (int half = 0; half < 2 && ok; ++half, ++ait) {
-                        const int a = ait % ASTAGES;
-                        if (!mbar_wait(&sm.act_full[a], (ait / ASTAGES) & 1, abort, ROLE_MMA)) { ok = false; break; }
-                        for (int hh = 0; hh < 4; ++hh) {
-                            const int h = 4 * half + hh;  // K step of the block = TMEM slot
-                            if (!mbar_wait(&sm.slot_full[h], it & 1, abort, ROLE_MMA)) { ok = false; break; }
-                            tc_fence_after();
+        // The whole warp walks the loop (converged, as tcgen05 issue wants it); the
+        // same elected lane issues every MMA and every commit that tracks them.
+        const uint32_t idesc = idesc_f8f6f4(BW, BT, /*A E5M2*/ 1u, /*B E4M3*/ 0u);
+        // descriptor of stage 0's first K slice; stage a and slice hh add their offsets
+        // (in 16-byte units) to the start-address field
+        const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(sm.act[0]));
+        int ait = 0, it = 0, tc = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tc) {
+            // the epilogue has read the previous tile's accumulator
+            if (!warp_wait(&sm.acc_empty, (tc & 1) ^ 1, abort, ROLE_MMA)) { ok = false; break; }
+            tc_fence_after();
+            for (int kb = 0; kb < num_kb && ok; ++kb, ++it) {
+                for (int half = 0; half < 2 && ok; ++half, ++ait) {
+                    const int a = ait % ASTAGES;
+                    if (!warp_wait(&sm.act_full[a], (ait / ASTAGES) & 1, abort, ROLE_MMA)) { ok = false; break; }
+                    for (int hh = 0; hh < 4; ++hh) {
+                        const int h = 4 * half + hh;  // K step of the block = TMEM slot
+                        if (!warp_wait(&sm.slot_full[h], it & 1, abort, ROLE_MMA)) { ok = false; break; }
+                        tc_fence_after();
+                        if (elect_one()) {
                             // B: the K = 32 slice of the 256 activation rows (128-byte swizzle)
                             const uint64_t bdesc = bdesc0 + (uint64_t)(a * (BT * 128 / 16) + hh * 2);
                             const uint32_t a0 = tmem + ACC_COLS + h * SLOT_COLS;
@@ -306,11 +308,16 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
                                 mma_f8f6f4_ts(tmem, a0 + i * 8, bdesc, idesc, (kb | h | i) != 0);
                             mma_commit(&sm.slot_empty[h]);
                         }
-                        if (ok) mma_commit(&sm.act_empty[a]);  // this stage's activations are read
+                        __syncwarp();
                     }
+                    if (ok && elect_one()) mma_commit(&sm.act_empty[a]);  // this stage's activations are read
+                    __syncwarp();
                 }
-                if (ok) mma_commit(&sm.acc_full);
             }
+            if (ok && elect_one()) mma_commit(&sm.acc_full);
+            __syncwarp();
+        }
+        if (elect_one()) {
             mma_commit(&sm.drain);
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&sm.drain, 0)) {
@@ -320,6 +327,7 @@ w4a8_kernel(const __grid_constant__ CUtensorMap tmA,   // E4M3 [M][K], box 128 B
                 }
             }
         }
+        __syncwarp();
     } else if (warp >= FIRST_CONV && warp < FIRST_CONV + CONV_WARPS) {
         // ------------------------------------------------------------ converters
         const int q = warp & 3;                      // TMEM lane quarter this warp may access
