@@ -495,8 +495,11 @@ nvfp4_status nvfp4_quantize_bf16(const void* X, int rows, int K, uint8_t* codes,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, q::quantize_bf16_kernel, static_cast<const __nv_bfloat16*>(X), rows,
-                           K, static_cast<const unsigned*>(amax), codes, scales, scales_packed, g_out);
+    // 256-bit loads when X starts on a 32-byte boundary (rows then do too: K % 16 == 0)
+    auto kern = reinterpret_cast<uintptr_t>(X) % 32 == 0 ? q::quantize_bf16_kernel<true>
+                                                          : q::quantize_bf16_kernel<false>;
+    e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(X), rows, K,
+                           static_cast<const unsigned*>(amax), codes, scales, scales_packed, g_out);
     if (e != cudaSuccess) return cuda_fail(e, "launching quantize_bf16_kernel");
     return ok();
 }

@@ -28,7 +28,7 @@ constexpr int AMAX_THREADS = 512;
 constexpr int TILE_ROWS = 128;   // one packed 128-row block
 constexpr int TILE_COLS = 256;   // 16 groups: four K = 64 steps
 constexpr int THREADS = 256;     // 8 warps x 16 rows
-constexpr int QB = 4;            // row segments of a warp in flight at once
+constexpr int QB = 4;            // row pairs of a warp in flight at once
 
 // max over |x| as BF16 magnitude bits (15 bits), into *amax_bits (atomic max)
 __global__ void __launch_bounds__(AMAX_THREADS)
@@ -104,10 +104,61 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&t)[8]) {
     return r;
 }
 
+// The sixteen BF16 values of one group, as eight words (element 2j in the low half
+// of word j).  V8: one 256-bit load (the row start is 32-byte aligned); otherwise two
+// 128-bit loads.  Streaming: X is read once more by nobody.
+template <bool V8>
+__device__ __forceinline__ void load_group(const __nv_bfloat16* p, uint32_t (&w)[8]) {
+    if constexpr (V8) {
+        asm("ld.global.cs.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+            : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+              "=r"(w[7])
+            : "l"(p));
+    } else {
+        const uint4 a = __ldcs(reinterpret_cast<const uint4*>(p));
+        const uint4 b = __ldcs(reinterpret_cast<const uint4*>(p) + 1);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    }
+}
+
+// a / b by Markstein's correction from y = RN(1/b), for b in [2^-60, 2^60] and
+// 0 <= a / b <= 2^68: q = RN(a*y), r = a - b*q (exact by FMA), RN(q + r*y).  That is
+// RN(a / b) whenever a >= 2^-100, where no step underflows; below that the result
+// can be off in its last (subnormal) places or be -0.
+__device__ __forceinline__ float div_markstein(float a, float b, float y) {
+    const float q = __fmul_rn(a, y);
+    const float r = __fmaf_rn(-b, q, a);
+    return __fmaf_rn(r, y, q);
+}
+
+// prmt.b32 in its generic mode: a selector nibble with bit 3 set fills the byte
+// with the sign (bit 7) of the selected source byte.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Eight codes (element 2j in the low nibble of byte j) with each sign bit set from
+// x's own sign, the eight BF16 values being w0 .. w3 (element 2j in the low half of
+// word j).  A correctly rounded x / den with den > 0 has x's sign, -0 and values that
+// round to zero included; the corrected quotient can lose that sign only where it
+// underflows, which is far below the smallest nonzero code.
+__device__ __forceinline__ uint32_t with_signs(uint32_t code, uint32_t w0, uint32_t w1, uint32_t w2,
+                                               uint32_t w3) {
+    const uint32_t a = prmt(w0, w1, 0xFDB9u);    // bytes 0x00/0xFF: signs of elements 0..3
+    const uint32_t b = prmt(w2, w3, 0xFDB9u);    // elements 4..7
+    const uint32_t even = prmt(a, b, 0x6420u);   // elements 0, 2, 4, 6
+    const uint32_t odd = prmt(a, b, 0x7531u);    // elements 1, 3, 5, 7
+    return (code & 0x77777777u) | (even & 0x08080808u) | (odd & 0x80808080u);
+}
+
 // One CTA: rows [128*blockIdx.x, +128) x columns [256*blockIdx.y, +256).
-// Warp w takes rows 16w .. 16w+15; lane l holds columns 8l .. 8l+7 of the row
-// (lanes 2j and 2j+1 make group j).
-__global__ void __launch_bounds__(THREADS)
+// One lane per 16-group: lanes 16h .. 16h+15 of warp w take the 16 groups of row
+// 16w + 2i + h (i = 0 .. 7), so a warp instruction covers two rows of the tile.
+template <bool V8>
+__global__ void __launch_bounds__(THREADS, 4)
 quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
                      const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
                      uint8_t* __restrict__ scales, uint8_t* __restrict__ scales_packed,
@@ -115,18 +166,22 @@ quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
     __shared__ uint32_t sc[TILE_ROWS][TILE_COLS / 64 + 1];  // [row][K=64 step] four scale bytes
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blockIdx.x * TILE_ROWS, c0 = blockIdx.y * TILE_COLS;
-    const int col = c0 + 8 * lane;
-    const bool col_ok = col < K;  // K % 16 == 0: a lane's 8 columns are all in or all out
+    const int gi = lane & 15, half = lane >> 4;  // group of the tile row; which row of the pair
+    const int col = c0 + 16 * gi;
+    const bool col_ok = col < K;  // K % 16 == 0: a group is all in or all out
 
-    // this warp's 16 row segments, QB at a time in flight before any is used
-    constexpr int RPW = TILE_ROWS / 8;  // rows per warp
-    uint4 vin[QB];
+    constexpr int PAIRS = TILE_ROWS / 16;  // row pairs per warp
+    uint32_t vin[QB][8];
     auto load_rows = [&](int i0) {
 #pragma unroll
         for (int i = 0; i < QB; ++i) {
-            const int row = r0 + warp * RPW + i0 + i;
-            vin[i] = make_uint4(0u, 0u, 0u, 0u);
-            if (col_ok && row < rows) vin[i] = __ldcs(reinterpret_cast<const uint4*>(X + (size_t)row * K + col));
+            const int row = r0 + warp * 16 + 2 * (i0 + i) + half;
+            if (col_ok && row < rows) {
+                load_group<V8>(X + (size_t)row * K + col, vin[i]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) vin[i][j] = 0u;
+            }
         }
     };
     // The first rows are read while the amax kernel before this one may still run
@@ -135,66 +190,71 @@ quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
     grid_dependency_wait();
     const float g = global_scale(__ldcg(amax_bits));
     const float d6 = __fmul_rn(6.0f, g);
+    const bool fast6 = d6 >= 0x1p-60f && d6 <= 0x1p60f;  // the same for the whole tensor
+    const float y6 = __frcp_rn(d6);
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = g;
+    uint8_t* scb = reinterpret_cast<uint8_t*>(&sc[0][0]);
 #pragma unroll 1
-    for (int i0 = 0; i0 < RPW; i0 += QB) {
+    for (int i0 = 0; i0 < PAIRS; i0 += QB) {
         if (i0 > 0) load_rows(i0);
 #pragma unroll
-    for (int i = 0; i < QB; ++i) {
-        const int rl = warp * RPW + i0 + i;
-        const int row = r0 + rl;
-        const bool ok = col_ok && row < rows;
-        const uint4 v = vin[i];
-        // group amax over the lane pair (integer max of the magnitude bits)
-        const unsigned a = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                                    __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-        unsigned m = max(a & 0xFFFFu, a >> 16);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        const float amax_b = __uint_as_float(m << 16);
-        const uint32_t sb = e4m3_satfinite(__fdiv_rn(amax_b, d6));
-        const float den = __fmul_rn(e4m3_value(sb), g);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float t[8];
-        // t = x / den, correctly rounded.  The divisor is shared by the group, so its
-        // correctly rounded reciprocal y is taken once and each quotient is finished by
-        // Markstein's correction (q = RN(x*y), r = x - den*q exactly by FMA,
-        // t = RN(q + r*y)), which gives RN(x/den) when no step under- or overflows:
-        // true for den in [2^-60, 2^60] (|t| stays below 7 by the choice of s).  Other
-        // groups, and den == 0, keep the plain division.
-        const bool fast = den >= 0x1p-60f && den <= 0x1p60f;
-        if (fast) {
-            // both halves of a word at once (packed f32x2 lanes, each one IEEE RN op)
-            const float y = __frcp_rn(den);
-            const uint64_t y2 = ((uint64_t)__float_as_uint(y) << 32) | __float_as_uint(y);
-            const uint64_t nd2 = ((uint64_t)__float_as_uint(-den) << 32) | __float_as_uint(-den);
+        for (int i = 0; i < QB; ++i) {
+            const int rl = warp * 16 + 2 * (i0 + i) + half;
+            const int row = r0 + rl;
+            const bool ok = col_ok && row < rows;
+            const uint32_t(&w)[8] = vin[i];
+            // group amax (integer max of the magnitude bits; they order like the values)
+            const unsigned a01 = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
+            const unsigned a23 = __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu);
+            const unsigned a45 = __vmaxu2(w[4] & 0x7FFF7FFFu, w[5] & 0x7FFF7FFFu);
+            const unsigned a67 = __vmaxu2(w[6] & 0x7FFF7FFFu, w[7] & 0x7FFF7FFFu);
+            const unsigned a = __vmaxu2(__vmaxu2(a01, a23), __vmaxu2(a45, a67));
+            const float amax_b = __uint_as_float(max(a & 0xFFFFu, a >> 16) << 16);
+            // s_b = E4M3(RN(amax_b / (6g))); amax_b <= amax makes the quotient <= 448
+            // (|.|: the corrected quotient may come out as -0 where it underflows; the
+            // scale byte is 0 there either way)
+            const float qs = fast6 ? fabsf(div_markstein(amax_b, d6, y6)) : __fdiv_rn(amax_b, d6);
+            const uint32_t sb = e4m3_satfinite(qs);
+            const float den = __fmul_rn(e4m3_value(sb), g);
+            float t[16];
+            // t = x / den, correctly rounded.  The divisor is shared by the group, so its
+            // correctly rounded reciprocal is taken once and each quotient is finished by
+            // Markstein's correction on packed f32x2 lanes (two elements per instruction,
+            // each lane one IEEE RN operation).  For den in [2^-60, 2^60] that is RN(x/den)
+            // wherever x / den >= 2^-3 in magnitude (every step stays normal; |t| < 7 by
+            // the choice of s); smaller quotients give a zero code whatever their last
+            // places, and with_signs gives it x's sign.  Other groups, and den == 0, keep
+            // the plain division.
+            if (den >= 0x1p-60f && den <= 0x1p60f) {
+                const float y = __frcp_rn(den);
+                const uint64_t y2 = ((uint64_t)__float_as_uint(y) << 32) | __float_as_uint(y);
+                const uint64_t nd2 = ((uint64_t)__float_as_uint(-den) << 32) | __float_as_uint(-den);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint64_t x2 = ((uint64_t)(w[j] & 0xFFFF0000u) << 32) | (uint64_t)(w[j] << 16);
-                const uint64_t q2 = mul_f32x2(x2, y2);
-                const uint64_t t2 = fma_f32x2(fma_f32x2(q2, nd2, x2), y2, q2);
-                t[2 * j] = __uint_as_float((uint32_t)t2);
-                t[2 * j + 1] = __uint_as_float((uint32_t)(t2 >> 32));
-            }
-        } else {
+                for (int j = 0; j < 8; ++j) {
+                    const uint64_t x2 = ((uint64_t)(w[j] & 0xFFFF0000u) << 32) | (uint64_t)(w[j] << 16);
+                    const uint64_t q2 = mul_f32x2(x2, y2);
+                    const uint64_t t2 = fma_f32x2(fma_f32x2(q2, nd2, x2), y2, q2);
+                    t[2 * j] = __uint_as_float((uint32_t)t2);
+                    t[2 * j + 1] = __uint_as_float((uint32_t)(t2 >> 32));
+                }
+            } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                // element e is half (e & 1) of word e >> 1
-                const uint32_t h = (e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16);
-                const float xe = __uint_as_float(h);
-                t[e] = den > 0.f ? __fdiv_rn(xe, den) : xe * 0.0f;
+                for (int e = 0; e < 16; ++e) {
+                    // element e is half (e & 1) of word e >> 1
+                    const uint32_t h = (e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16);
+                    const float xe = __uint_as_float(h);
+                    t[e] = den > 0.f ? __fdiv_rn(xe, den) : xe * 0.0f;
+                }
             }
+            const float(&tlo)[8] = *reinterpret_cast<const float(*)[8]>(&t[0]);
+            const float(&thi)[8] = *reinterpret_cast<const float(*)[8]>(&t[8]);
+            if (ok)
+                *reinterpret_cast<uint2*>(codes + (size_t)row * (K / 2) + col / 2) =
+                    make_uint2(with_signs(e2m1x8(tlo), w[0], w[1], w[2], w[3]),
+                               with_signs(e2m1x8(thi), w[4], w[5], w[6], w[7]));
+            // the group's scale byte (group gi of the row is byte gi of the row's words)
+            scb[rl * (TILE_COLS / 64 + 1) * 4 + gi] = ok ? (uint8_t)sb : (uint8_t)0;
         }
-        const uint32_t out = e2m1x8(t);
-        if (ok) *reinterpret_cast<uint32_t*>(codes + (size_t)row * (K / 2) + col / 2) = out;
-        // the group's scale byte: lane 2j holds group j; gather four groups (one K = 64
-        // step) into one word in shared memory
-        const uint32_t b0 = __shfl_sync(0xffffffffu, sb, (lane & ~7) + 0);
-        const uint32_t b1 = __shfl_sync(0xffffffffu, sb, (lane & ~7) + 2);
-        const uint32_t b2 = __shfl_sync(0xffffffffu, sb, (lane & ~7) + 4);
-        const uint32_t b3 = __shfl_sync(0xffffffffu, sb, (lane & ~7) + 6);
-        const uint32_t word = row < rows ? (b0 | (b1 << 8) | (b2 << 16) | (b3 << 24)) : 0u;
-        if ((lane & 7) == 0) sc[rl][lane >> 3] = col_ok ? word : 0u;
-    }
     }
     __syncthreads();
 

@@ -1,12 +1,13 @@
-"""Every output element of the full-size workloads against the FP64 oracle.
+"""Every output element of the full-size workloads against the oracle.
 
 The FFN-down product (4096 x 5376 x 14336) through every entry point that computes
 it -- the plain-scale single-SM kernel, the SM-pair kernel with whole tiles and with
 the last waves cut between pairs (the benchmark's launch), and the exact FP8 path --
 the W4A8 product on the same shape, and the 8-expert grouped product (8192 routed
 tokens, 14336 x 4096 experts) through the host-planned and the device-offset entry
-points.  Each oracle result is computed once per session and shared; each
-comparison asserts that all M*N outputs were compared."""
+points, and the activation quantiser on the FFN-down activations.  Each oracle
+result is computed once per session and shared; each comparison asserts that all
+outputs were compared."""
 import functools
 
 import numpy as np
@@ -109,3 +110,26 @@ def test_grouped_every_output(path):
             c1 = min(r1, c0 + CHUNK)
             acc.add(y[c0:c1].float().cpu().numpy().astype(np.float64), refs[e][c0 - r0:c1 - r0])
     acc.finish(t.M * t.N)
+
+
+def test_quantiser_every_element_full_size():
+    """The FFN-down activations (4096 x 14336 BF16): every code, every plain and packed
+    scale byte and g, bit for bit against the oracle's quantiser.  The tensor holds a
+    few -0 inputs inside groups with a nonzero scale, whose codes must keep the sign."""
+    from oracle import quantize as oq
+    from parity import packed_reference
+    t = wl.activations_bf16()
+    bits = t.A_bf16.view(np.uint16)
+    x = _dev(bits.view(np.int16)).view(torch.bfloat16)
+    codes, s, sp, g = nv.nvfp4_quantize_bf16(x, plain=True, packed=True)
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    rc, rs, rg = oq.quantize_nvfp4_bf16(bits)
+    assert float(g.cpu().numpy()[0]) == float(rg)
+    got = codes.cpu().numpy()
+    assert got.shape == rc.shape
+    bad = np.argwhere(got != rc)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first {bad[:5]}"
+    assert np.array_equal(s.cpu().numpy(), rs)
+    ref = packed_reference(rs, bits.shape[1])
+    assert np.array_equal(sp.cpu().numpy()[:ref.size], ref)

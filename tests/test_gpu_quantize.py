@@ -59,8 +59,9 @@ def test_plain_only_and_packed_only():
 
 
 def test_special_values():
-    """Zero rows and blocks, -0, tiny values that give E4M3-subnormal and zero block
-    scales, the BF16 extremes, and values at E2M1 midpoints of their block."""
+    """Zero rows and blocks, -0 (alone and inside a block with a nonzero scale), tiny
+    values that give E4M3-subnormal and zero block scales or quotients that underflow,
+    the BF16 extremes, and values at E2M1 midpoints of their block."""
     rng = np.random.default_rng(2)
     x = rng.standard_normal((8, 256)).astype(np.float32)
     x[0] = 0.0                                  # a zero row
@@ -69,6 +70,10 @@ def test_special_values():
     x[3, :16] = np.float32(3e38)                # the tensor amax near the BF16 maximum
     x[3, 16:32] = -np.float32(3e38)
     x[4, 32:48] = np.float32(1e-5) * rng.standard_normal(16)   # subnormal E4M3 scales
+    x[6, 16:32] = rng.standard_normal(16)
+    x[6, 17] = -0.0                             # -0 and quotients that underflow, in a
+    x[6, 20] = -1e-38                           # group with a nonzero scale: codes -0
+    x[6, 21] = 1e-38
     base = np.float32(2.0 ** -3)
     x[5, :16] = base * np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -0.25, -0.75,
                                  -1.25, -1.75, -2.5, -3.5, -5, 0], np.float32)
@@ -156,3 +161,55 @@ def test_every_element_bit_exact_over_distributions(dist):
         x = (rng.standard_normal((rows, K)) *
              np.exp2(rng.integers(-100, 100, size=(rows, K // 16))).repeat(16, axis=1)).astype(np.float32)
     _expect_equal(_bits(x), K)
+
+
+def _groups_with_maxima(maxima, K, rng):
+    """One 16-group per entry of `maxima` (BF16 magnitude bits), row-major over rows of
+    K columns, zero-padded: each group holds its maximum once (random place and sign)
+    and 15 magnitudes drawn uniformly from [0, maximum]."""
+    n = maxima.size
+    gpr = K // 16
+    rows = -(-n // gpr)
+    mx = np.zeros(rows * gpr, np.uint32)
+    mx[:n] = maxima
+    mags = np.floor(rng.random((rows * gpr, 16)) * (mx[:, None] + 1)).astype(np.uint32)
+    mags = np.minimum(mags, mx[:, None])
+    mags[np.arange(rows * gpr), rng.integers(0, 16, rows * gpr)] = mx
+    sign = rng.integers(0, 2, (rows * gpr, 16)).astype(np.uint32) << 15
+    return ((mags | sign).astype(np.uint16)).reshape(rows, K)
+
+
+@pytest.mark.parametrize("top", [0x7F7F, 0x4700, 0x3F80, 0x2D00, 0x2000, 0x1E00, 0x0400, 0x0100])
+def test_every_bf16_group_maximum_bit_exact(top):
+    """Every BF16 magnitude up to the tensor's maximum `top` is one group's maximum, so
+    each scale quotient amax_b / (6 g) the tensor can produce is taken once and compared
+    with the oracle's.  The maxima span both sides of the kernel's range test on 6g
+    (448 * 2^-60 and 448 * 2^60 lie between the chosen tops), subnormal group maxima
+    included."""
+    rng = np.random.default_rng(top)
+    maxima = np.arange(0, top + 1, dtype=np.uint32)
+    rng.shuffle(maxima)
+    K = 1024
+    bits = _groups_with_maxima(maxima, K, rng)
+    _expect_equal(bits, K)
+
+
+def test_unaligned_tensor_takes_the_128bit_loads():
+    """A tensor that starts 16 bytes past a 32-byte boundary is read with 128-bit loads
+    instead of 256-bit ones; the results are the same bytes."""
+    rng = np.random.default_rng(77)
+    rows, K = 300, 1024
+    bits = _bits(rng.standard_normal((rows, K)).astype(np.float32))
+    base = torch.zeros(rows * K + 8, dtype=torch.int16, device="cuda")
+    base[8:] = torch.from_numpy(bits.view(np.int16).reshape(-1)).cuda()
+    x = base[8:].view(torch.bfloat16).view(rows, K)
+    assert x.data_ptr() % 32 == 16
+    codes, s, sp, g = nv.nvfp4_quantize_bf16(x, plain=True, packed=True)
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    rc, rs, rg = oq.quantize_nvfp4_bf16(bits)
+    assert float(g.cpu().numpy()[0]) == float(rg)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(s.cpu().numpy(), rs)
+    ref = packed_reference(rs, K)
+    assert np.array_equal(sp.cpu().numpy()[:ref.size], ref)
