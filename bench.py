@@ -612,6 +612,11 @@ def run_ours(args):
     gstarts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     gends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with ClockSampler(dev.index) as clk:
+        # `value` times whole steps with nothing between their kernels (an event recorded
+        # between the scale packing and the product would stop the product's launch from
+        # overlapping the packing), or the graph replay.  Those steps alternate with the
+        # steps that carry the per-kernel events, so that both see the same clocks and
+        # temperature over a long run.
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
@@ -622,12 +627,7 @@ def run_ours(args):
             else:
                 step()
             ends[i].record(stream)
-        torch.cuda.synchronize(dev)
-        if graph is not None or mids is not None:
-            # `value`: whole steps with nothing between their kernels (an event recorded
-            # between the scale packing and the product would stop the product's launch
-            # from overlapping the packing), or the graph replay
-            for i in range(args.steps):
+            if graph is not None or mids is not None:
                 flush.zero_()
                 gstarts[i].record(stream)
                 if graph is not None:
@@ -635,7 +635,7 @@ def run_ours(args):
                 else:
                     step()
                 gends[i].record(stream)
-            torch.cuda.synchronize(dev)
+        torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     nv.nvfp4_check_device_error(stream)
