@@ -225,8 +225,9 @@ NVFP4_API nvfp4_status nvfp4_quantize_bf16(const void* X_bf16, int rows, int K, 
  * pages; it is a convenience of this library.
  *   - It allocates nothing and calls no allocating routine.  Every GPU that
  *     loads the library holds the 256-byte array until the process exits.
- *   - The first call on a device looks up the array's device address (once per
- *     device); make that first call before any stream capture.
+ *   - Every call looks up the array's address in the current context (a query
+ *     that allocates nothing); make the first call on a device before any
+ *     stream capture, since it may load the library's device code.
  *   - Every call uses the same array; the call clears the part it needs, but
  *     calls whose work overlaps on the GPU (other streams, other threads) race
  *     on it and must be ordered by the caller.
