@@ -180,3 +180,22 @@ def test_dequantised_error_within_half_a_code_step():
     x = oq.bf16_to_f32(bits).astype(np.float64)
     half_step = np.array([0.25, 0.25, 0.25, 0.25, 0.5, 0.5, 1.0, 1.0])[codes & 7]
     assert np.all(np.abs(x - mag * sg) <= half_step * sg * (1 + 2.0 ** -20) + 1e-30)
+
+
+def test_signed_zero_codes_inside_a_live_block():
+    """In a block with a nonzero scale, -0 and a negative value whose quotient rounds to
+    zero both give the code -0 (nibble 8), their positive twins +0: the code is the
+    signed E2M1 rounding of the IEEE quotient, and x / (s g) keeps x's sign."""
+    x = np.zeros(16, np.float32)
+    x[0] = 1.0                      # the block maximum: a nonzero scale
+    x[1] = -0.0
+    x[2] = np.float32(-1e-38)       # BF16 subnormal; the quotient underflows to -0
+    x[3] = np.float32(1e-38)
+    x[4] = np.float32(-0.01)        # rounds to zero against 1/6 of the max
+    bits = to_bf16_bits(x[None, :])
+    p, s, g = oq.quantize_nvfp4_bf16(bits)
+    assert s[0, 0] != 0
+    nib = [(int(p[0, e >> 1]) >> (4 * (e & 1))) & 0xF for e in range(16)]
+    assert nib[1] == 8 and nib[2] == 8 and nib[4] == 8
+    assert nib[3] == 0 and all(n == 0 for n in nib[5:])
+    assert nib[0] != 0
