@@ -80,8 +80,8 @@ WORKLOADS = {
     "quantize": dict(path="quantize", bound="hbm",
                      desc="NVFP4 quantiser of the FFN-down activations, BF16 4096x14336"),
     "moe": dict(path="moe", bound="tensor",
-                desc="MoE layer from BF16 tokens (quantise, route, permute, grouped W4A4, "
-                     "combine), 8 experts [14336,4096], 8192 tokens"),
+                desc="MoE layer from BF16 tokens (route, quantise into the experts' row order, "
+                     "grouped W4A4, combine), 8 experts [14336,4096], 8192 tokens"),
 }
 
 
@@ -504,13 +504,11 @@ def run_ours(args):
         sw_packed = nv.nvfp4_pack_scales_grouped(Ws_d.view(E * N, K // 16),
                                                  [e * N for e in range(E + 1)], K, stream=stream)
         q_ws = torch.empty(16, dtype=torch.uint8, device=dev)
-        codes_b = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
-        scales_b = torch.empty((M, K // 16), dtype=torch.uint8, device=dev)
         g_b = torch.empty(4, dtype=torch.float32, device=dev)
         route_ws = torch.empty(nv.load_library().nvfp4_moe_route_workspace_bytes(M, E),
                                dtype=torch.uint8, device=dev)
-        gc_b = torch.empty_like(codes_b)
-        gs_b = torch.empty_like(scales_b)
+        gc_b = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)    # codes, experts' order
+        gs_b = torch.empty((M, K // 16), dtype=torch.uint8, device=dev)   # scales, experts' order
         ones = torch.ones((M, 1), dtype=torch.float32, device=dev)
 
         sa_b = torch.empty(nv.load_library().nvfp4_grouped_scale_layout_bytes_bound(M, E, K),
@@ -525,21 +523,20 @@ def run_ours(args):
                 if stages is not None:
                     stages[i].record(s)
             mark(0)
-            nv.nvfp4_quantize_bf16(dv[0].view(torch.bfloat16), plain=True, packed=False,
-                                   workspace=q_ws, stream=s, out=(codes_b, scales_b, None, g_b))
-            mark(1)
             off, dest, src = nv.moe_route(dv[1], E, workspace=route_ws, stream=s)
+            mark(1)
+            # the quantiser writes each token's codes and scales straight to its row in
+            # the experts' order (the dispatch permutation, fused)
+            nv.nvfp4_quantize_bf16_routed(dv[0].view(torch.bfloat16), dest, 1, workspace=q_ws,
+                                          stream=s, out=(gc_b, gs_b, g_b))
             mark(2)
-            nv.moe_permute_rows(codes_b, src, 1, out=gc_b, stream=s)
-            nv.moe_permute_rows(scales_b, src, 1, out=gs_b, stream=s)
-            mark(3)
             sched = nv.GroupedSchedule(off, E, M, N, K, gws, gA=g_b[:1], stream=s)
             sched.pack(gs_b, out=sa_b, stream=s)
-            mark(4)
+            mark(3)
             # top-1: the combine (weight, then each row to its token) is fused into the
             # grouped product's epilogue, so the expert-order rows never reach memory
             sched.gemm_combine(gc_b, sa_b, Wc_d, sw_packed, src, M, weights=ones, out=Y, stream=s)
-            mark(5)
+            mark(4)
     elif path == "w4a8":
         def step():
             nv.gemm_nvfp4_w4a8(dv[0], wl_.gA, dv[1], dv[2], wl_.W.g, out=Y, stream=stream)
@@ -567,7 +564,7 @@ def run_ours(args):
         def plain_step():
             nv.gemm_nvfp4_w4a4(dv[0], dv[1], wl_.A.g, dv[2], dv[3], wl_.W.g, out=Y, stream=stream)
     launches_per_step = {"w4a16": (M + 15) // 16, "w4a4": 2, "grouped": 2, "quantize": 2,
-                         "moe": 8}.get(path, 1)
+                         "moe": 6}.get(path, 1)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -747,12 +744,11 @@ def run_ours(args):
                  "plain_scale_entry_ms": statistics.median(plain),
                  "plain_scale_entry_tflops": flops / (statistics.median(plain) * 1e-3) / 1e12}
     if stage_ev is not None:
-        names = ["quantize", "route", "permute", "schedule_and_pack", "grouped_gemm_and_combine"]
+        names = ["route", "quantize_dispatched", "schedule_and_pack", "grouped_gemm_and_combine"]
         med = {n: statistics.median(ev[j].elapsed_time(ev[j + 1]) for ev in stage_ev) * 1e3
                for j, n in enumerate(names)}
         kern_s = med["grouped_gemm_and_combine"] * 1e-6
-        extra = {"stage_us": med,
-                 "permute_gbs": 2 * M * (K // 2 + K // 16) / (med["permute"] * 1e-6) / 1e9}
+        extra = {"stage_us": med}
     kernel_name = {"w4a4": "w4a4_pair_kernel", "via_fp8": "via_fp8_kernel", "w4a8": "w4a8_kernel",
                    "moe": "grouped_pair_kernel",
                    "w4a16": "w4a16_ldg_kernel", "grouped": "grouped_pair_kernel",

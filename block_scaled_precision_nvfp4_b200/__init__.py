@@ -30,7 +30,8 @@ __all__ = [
     "nvfp4_pack_scales", "nvfp4_prepare_scales", "nvfp4_workspace_size", "Op",
     "gemm_nvfp4_w4a4_packed", "nvfp4_w4a4_packed_workspace_bytes", "w4a4_packed_workspace",
     "nvfp4_grouped_scale_layout_bytes", "nvfp4_pack_scales_grouped",
-    "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "nvfp4_fp4_fallback",
+    "gemm_nvfp4_w4a4_grouped_packed", "nvfp4_quantize_bf16", "nvfp4_quantize_bf16_routed",
+    "nvfp4_fp4_fallback",
     "nvfp4_node_exec", "moe_route", "moe_permute_rows", "moe_combine", "GroupedSchedule",
     "C_FUNCTIONS",
 ]
@@ -131,6 +132,7 @@ C_FUNCTIONS = {
                                                           _I, _I, _I, _P]),
     "nvfp4_quantize_bf16": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _Z, _P]),
     "nvfp4_quantize_bf16_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _P]),
+    "nvfp4_quantize_bf16_routed": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P, _Z, _P]),
 }
 
 _lock = threading.Lock()
@@ -334,6 +336,45 @@ def nvfp4_quantize_bf16(x, plain=True, packed=True, workspace=None, stream=None,
                                  workspace.data_ptr(),
                                  workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
     return codes, scales, sp, g[:1]
+
+
+def nvfp4_quantize_bf16_routed(x, dest, k=1, workspace=None, stream=None, out=None):
+    """nvfp4_quantize_bf16 writing token row r's codes and plain scales to rows
+    dest[r*k + j] (j < k): the quantised rows in an MoE dispatch's order.
+
+    `dest` is the int32 [rows*k] CUDA tensor nvfp4_moe_route returns.  Returns (codes
+    uint8 [rows*k, K/2], scales uint8 [rows*k, K/16], g: 1-element float32 CUDA tensor);
+    `out`, if given, is such a tuple of preallocated tensors."""
+    torch = _torch()
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise TypeError("x must be a 2-D torch.Tensor")
+    rows, K = x.shape
+    k = int(k)
+    px = _dev_tensor(x, torch.bfloat16, (rows, K), "x")
+    pd = _dev_tensor(dest, torch.int32, (rows * k,), "dest")
+    dev = x.device
+    if out is not None:
+        codes, scales, g = out
+    else:
+        codes = torch.empty((rows * k, K // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((rows * k, K // 16), dtype=torch.uint8, device=dev)
+        g = torch.empty(4, dtype=torch.float32, device=dev)
+    _dev_tensor(codes, torch.uint8, (rows * k, K // 2), "codes")
+    _dev_tensor(scales, torch.uint8, (rows * k, K // 16), "scales")
+    if g.dtype != torch.float32 or not g.is_cuda or g.numel() < 1:
+        raise ValueError("g must be a CUDA float32 tensor")
+    lib = load_library()
+    nws = int(lib.nvfp4_quantize_workspace_bytes())
+    if workspace is None:
+        workspace = torch.empty(nws, dtype=torch.uint8, device=dev)
+    if (not isinstance(workspace, torch.Tensor) or not workspace.is_cuda
+            or not workspace.is_contiguous() or workspace.numel() * workspace.element_size() < nws):
+        raise ValueError(f"workspace must be a contiguous CUDA tensor of >= {nws} bytes")
+    _err(lib.nvfp4_quantize_bf16_routed(px, rows, K, pd, k, codes.data_ptr(), scales.data_ptr(),
+                                        g.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream_ptr(stream)))
+    return codes, scales, g[:1]
 
 
 def nvfp4_w4a4_packed_workspace_bytes(M, N, K, max_pairs=0):

@@ -436,9 +436,12 @@ nvfp4_status nvfp4_pack_scales(const uint8_t* s_plain, int rows, int K, uint8_t*
 // ------------------------------------------------------------------------- quantiser
 size_t nvfp4_quantize_workspace_bytes(void) { return NVFP4_QUANTIZE_WORKSPACE_BYTES; }
 
-nvfp4_status nvfp4_quantize_bf16(const void* X, int rows, int K, uint8_t* codes, uint8_t* scales,
-                                 uint8_t* scales_packed, float* g_out, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
+namespace {
+// The quantiser's checks and launches; dest == nullptr writes row r to row r,
+// otherwise to rows dest[r k + j].
+nvfp4_status quantize_bf16_impl(const void* X, int rows, int K, uint8_t* codes, uint8_t* scales,
+                                uint8_t* scales_packed, float* g_out, void* workspace,
+                                size_t workspace_bytes, void* stream, const int32_t* dest, int k) {
     namespace q = nvfp4::quant;
     if (rows < 0) return fail(NVFP4_ERR_INVALID_ARG, "rows must be >= 0 (got %d)", rows);
     if (K < 16 || K % 16 != 0)
@@ -496,12 +499,35 @@ nvfp4_status nvfp4_quantize_bf16(const void* X, int rows, int K, uint8_t* codes,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // 256-bit loads when X starts on a 32-byte boundary (rows then do too: K % 16 == 0)
-    auto kern = reinterpret_cast<uintptr_t>(X) % 32 == 0 ? q::quantize_bf16_kernel<true>
-                                                          : q::quantize_bf16_kernel<false>;
+    const bool v8 = reinterpret_cast<uintptr_t>(X) % 32 == 0;
+    auto kern = dest ? (v8 ? q::quantize_bf16_kernel<true, true> : q::quantize_bf16_kernel<false, true>)
+                     : (v8 ? q::quantize_bf16_kernel<true, false> : q::quantize_bf16_kernel<false, false>);
     e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(X), rows, K,
-                           static_cast<const unsigned*>(amax), codes, scales, scales_packed, g_out);
+                           static_cast<const unsigned*>(amax), codes, scales, scales_packed, g_out,
+                           dest, k);
     if (e != cudaSuccess) return cuda_fail(e, "launching quantize_bf16_kernel");
     return ok();
+}
+}  // namespace
+
+nvfp4_status nvfp4_quantize_bf16(const void* X, int rows, int K, uint8_t* codes, uint8_t* scales,
+                                 uint8_t* scales_packed, float* g_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    return quantize_bf16_impl(X, rows, K, codes, scales, scales_packed, g_out, workspace,
+                              workspace_bytes, stream, nullptr, 1);
+}
+
+nvfp4_status nvfp4_quantize_bf16_routed(const void* X, int rows, int K, const int32_t* dest, int k,
+                                        uint8_t* codes, uint8_t* scales, float* g_out,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (k < 1 || k > 8) return fail(NVFP4_ERR_INVALID_ARG, "k must be in [1, 8] (got %d)", k);
+    if (!scales) return fail(NVFP4_ERR_INVALID_ARG, "the routed quantiser writes plain scales: null scales");
+    if (rows > 0 && !dest) return fail(NVFP4_ERR_INVALID_ARG, "null dest");
+    if (dest && reinterpret_cast<uintptr_t>(dest) % 4 != 0)
+        return fail(NVFP4_ERR_MISALIGNED, "dest must be 4-byte aligned");
+    if ((long long)rows * k > INT32_MAX) return fail(NVFP4_ERR_INVALID_ARG, "rows * k too large");
+    return quantize_bf16_impl(X, rows, K, codes, scales, nullptr, g_out, workspace, workspace_bytes,
+                              stream, rows > 0 ? dest : nullptr, k);
 }
 
 // ------------------------------------------------------------------------- quantiser without

@@ -157,12 +157,16 @@ __device__ __forceinline__ uint32_t with_signs(uint32_t code, uint32_t w0, uint3
 // One CTA: rows [128*blockIdx.x, +128) x columns [256*blockIdx.y, +256).
 // One lane per 16-group: lanes 16h .. 16h+15 of warp w take the 16 groups of row
 // 16w + 2i + h (i = 0 .. 7), so a warp instruction covers two rows of the tile.
-template <bool V8>
+// ROUTED: row r's codes and plain scales go to rows dest[r k + j] (j < k) of the
+// outputs instead of row r, which is the row permutation of an MoE dispatch done as
+// the rows are written (no packed scales then); a destination outside [0, rows k)
+// (-1: a pair the route placed nowhere) is skipped.
+template <bool V8, bool ROUTED>
 __global__ void __launch_bounds__(THREADS, 4)
 quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
                      const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
                      uint8_t* __restrict__ scales, uint8_t* __restrict__ scales_packed,
-                     float* __restrict__ g_out) {
+                     float* __restrict__ g_out, const int32_t* __restrict__ dest, int k) {
     __shared__ uint32_t sc[TILE_ROWS][TILE_COLS / 64 + 1];  // [row][K=64 step] four scale bytes
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blockIdx.x * TILE_ROWS, c0 = blockIdx.y * TILE_COLS;
@@ -248,10 +252,20 @@ quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
             }
             const float(&tlo)[8] = *reinterpret_cast<const float(*)[8]>(&t[0]);
             const float(&thi)[8] = *reinterpret_cast<const float(*)[8]>(&t[8]);
-            if (ok)
-                *reinterpret_cast<uint2*>(codes + (size_t)row * (K / 2) + col / 2) =
-                    make_uint2(with_signs(e2m1x8(tlo), w[0], w[1], w[2], w[3]),
-                               with_signs(e2m1x8(thi), w[4], w[5], w[6], w[7]));
+            if (ok) {
+                const uint2 cv = make_uint2(with_signs(e2m1x8(tlo), w[0], w[1], w[2], w[3]),
+                                            with_signs(e2m1x8(thi), w[4], w[5], w[6], w[7]));
+                if (ROUTED) {
+                    for (int j = 0; j < k; ++j) {
+                        // a pair the route placed nowhere (-1) is skipped
+                        const int d = __ldg(dest + (size_t)row * k + j);
+                        if ((unsigned)d < (unsigned)(rows * k))
+                            *reinterpret_cast<uint2*>(codes + (size_t)d * (K / 2) + col / 2) = cv;
+                    }
+                } else {
+                    *reinterpret_cast<uint2*>(codes + (size_t)row * (K / 2) + col / 2) = cv;
+                }
+            }
             // the group's scale byte (group gi of the row is byte gi of the row's words)
             scb[rl * (TILE_COLS / 64 + 1) * 4 + gi] = ok ? (uint8_t)sb : (uint8_t)0;
         }
@@ -265,18 +279,22 @@ quantize_bf16_kernel(const __nv_bfloat16* __restrict__ X, int rows, int K,
             const int rl = idx >> 2, ks = idx & 3, row = r0 + rl;
             const int g0 = c0 / 16 + 4 * ks;  // first group of the word
             if (row < rows && g0 < K / 16) {
-                uint8_t* dst = scales + (size_t)row * (K / 16) + g0;
                 const uint32_t wv = sc[rl][ks];
                 const int n = min(4, K / 16 - g0);
-                if (n == 4 && (K / 16) % 4 == 0) {
-                    *reinterpret_cast<uint32_t*>(dst) = wv;  // 4-byte aligned
-                } else {
-                    for (int b = 0; b < n; ++b) dst[b] = (uint8_t)(wv >> (8 * b));
+                for (int j = 0; j < (ROUTED ? k : 1); ++j) {
+                    const int drow = ROUTED ? __ldg(dest + (size_t)row * k + j) : row;
+                    if (ROUTED && (unsigned)drow >= (unsigned)(rows * k)) continue;
+                    uint8_t* dst = scales + (size_t)drow * (K / 16) + g0;
+                    if (n == 4 && (K / 16) % 4 == 0) {
+                        *reinterpret_cast<uint32_t*>(dst) = wv;  // 4-byte aligned
+                    } else {
+                        for (int b = 0; b < n; ++b) dst[b] = (uint8_t)(wv >> (8 * b));
+                    }
                 }
             }
         }
     }
-    if (scales_packed && K % 64 == 0) {
+    if (!ROUTED && scales_packed && K % 64 == 0) {
         // packed[rb][ks][i][j][t] = s[128 rb + 32 j + i][4 ks + t]: this tile's nks atoms,
         // contiguous, one 16-byte line (i) per thread and step
         const int ksteps = K / 64, ks0 = c0 / 64;

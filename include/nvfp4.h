@@ -238,6 +238,26 @@ NVFP4_API nvfp4_status nvfp4_quantize_bf16_noalloc(const void* X_bf16, int rows,
                                                    uint8_t* scales_packed, float* g_out,
                                                    void* stream);
 
+/* nvfp4_quantize_bf16 with the rows written in an MoE dispatch's order: the
+ * quantisation of token row r (the same codes, scale bytes and g as the plain
+ * call) is written to output rows dest[r*k + j] for j < k, so that an MoE layer
+ * needs no separate permutation of the quantised rows before its grouped
+ * product (page 2, the FlashInfer swapab_cutedsl_megakernel skill doc, Layout:
+ * each expert's tokens as one contiguous block of rows).
+ *   dest    device, [rows*k] int32, the destination row of each (token, slot),
+ *           as nvfp4_moe_route writes it; a value outside [0, rows*k) (the
+ *           route's -1 for a pair with an out-of-range expert id) writes
+ *           nothing, and output rows no pair lands on are left untouched
+ *   k       slots per token, 1..8
+ *   codes   device, [rows*k][K/2];  scales  device, [rows*k][K/16] (required)
+ * The packed scale layout is not written (an MoE layer packs per expert).
+ * Other arguments, alignment, errors and determinism as nvfp4_quantize_bf16;
+ * dest must be 4-byte aligned. */
+NVFP4_API nvfp4_status nvfp4_quantize_bf16_routed(const void* X_bf16, int rows, int K,
+                                                  const int32_t* dest, int k, uint8_t* codes,
+                                                  uint8_t* scales, float* g_out, void* workspace,
+                                                  size_t workspace_bytes, void* stream);
+
 /* gemm_nvfp4_w4a4 with both scale matrices already packed
  * (nvfp4_pack_scales / nvfp4_prepare_scales); the same product, module doc
  * bullet 1, the NVFP4 row.  Runs on pairs of SMs (tcgen05 cta_group::2, 256 x 256

@@ -213,3 +213,64 @@ def test_unaligned_tensor_takes_the_128bit_loads():
     assert np.array_equal(s.cpu().numpy(), rs)
     ref = packed_reference(rs, K)
     assert np.array_equal(sp.cpu().numpy()[:ref.size], ref)
+
+
+@pytest.mark.parametrize("rows,K,E,k", [(1000, 2048, 8, 1), (300, 512, 4, 2), (257, 4160, 8, 1),
+                                         (64, 96, 3, 3)])
+def test_routed_quantiser_writes_the_dispatch_order(rows, K, E, k):
+    """nvfp4_quantize_bf16_routed with the route's dest equals the plain quantiser
+    followed by the route's row permutation (out[dest[p]] = row p // k), bit for bit,
+    with the same g."""
+    rng = np.random.default_rng(rows + K + E + k)
+    bits = _bits(rng.standard_normal((rows, K)).astype(np.float32) * np.float32(3.0))
+    x = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    ids = torch.from_numpy(rng.integers(0, E, size=(rows, k)).astype(np.int32)).cuda()
+    off, dest, src = nv.moe_route(ids, E)
+    codes, scales, g = nv.nvfp4_quantize_bf16_routed(x, dest, k)
+    rc, rs, _, rg = nv.nvfp4_quantize_bf16(x, plain=True, packed=False)
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    assert float(g.cpu()[0]) == float(rg.cpu()[0])
+    d = dest.cpu().numpy()
+    assert sorted(d.tolist()) == list(range(rows * k))
+    rows_of = np.arange(rows * k) // k
+    want_c = np.empty((rows * k, K // 2), np.uint8)
+    want_s = np.empty((rows * k, K // 16), np.uint8)
+    want_c[d] = rc.cpu().numpy()[rows_of]
+    want_s[d] = rs.cpu().numpy()[rows_of]
+    assert np.array_equal(codes.cpu().numpy(), want_c)
+    assert np.array_equal(scales.cpu().numpy(), want_s)
+
+
+def test_routed_quantiser_skips_pairs_placed_nowhere():
+    """A destination outside [0, rows k) (the route's -1) writes nothing: that output
+    row keeps what was there, and every other row is the quantised source row."""
+    rng = np.random.default_rng(11)
+    rows, K, k = 96, 256, 2
+    bits = _bits(rng.standard_normal((rows, K)).astype(np.float32))
+    x = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    d = rng.permutation(rows * k).astype(np.int32)
+    hole = int(d[7])
+    d[7] = -1
+    dest = torch.from_numpy(d).cuda()
+    codes = torch.full((rows * k, K // 2), 0xAB, dtype=torch.uint8, device="cuda")
+    scales = torch.full((rows * k, K // 16), 0xCD, dtype=torch.uint8, device="cuda")
+    g = torch.empty(4, dtype=torch.float32, device="cuda")
+    nv.nvfp4_quantize_bf16_routed(x, dest, k, out=(codes, scales, g))
+    rc, rs, _, _ = nv.nvfp4_quantize_bf16(x, plain=True, packed=False)
+    torch.cuda.synchronize()
+    nv.nvfp4_check_device_error()
+    c, s = codes.cpu().numpy(), scales.cpu().numpy()
+    assert np.all(c[hole] == 0xAB) and np.all(s[hole] == 0xCD)
+    rc, rs = rc.cpu().numpy(), rs.cpu().numpy()
+    for p in range(rows * k):
+        if d[p] >= 0:
+            assert np.array_equal(c[d[p]], rc[p // k]) and np.array_equal(s[d[p]], rs[p // k])
+
+
+def test_routed_quantiser_argument_errors():
+    x = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
+    dest = torch.arange(4 * 9, dtype=torch.int32, device="cuda")
+    with pytest.raises(nv.NvFp4Error) as e:   # k above 8
+        nv.nvfp4_quantize_bf16_routed(x, dest, 9)
+    assert e.value.status == nv.Status.INVALID_ARG
