@@ -1,8 +1,9 @@
 // quantize_kernel.cuh -- BF16 activations -> NVFP4 (E2M1 codes, E4M3 group
 // scales, FP32 per-tensor scale): the step ahead of the W4A4 matmul.
 //
-// Two-level recipe of the FFN-down workload ("per-16 scale = amax/6 rounded to
-// E4M3 and a per-tensor FP32 scale = tensor amax/(6*448)"), every step an IEEE
+// Two-level recipe of the FFN-down workload: each run of 16 elements gets an E4M3
+// scale from its largest magnitude over 6, taken relative to an FP32 per-tensor
+// scale from the tensor's largest magnitude over 6 x 448.  Every step is an IEEE
 // FP32 operation rounded to nearest even, in this order:
 //     g      = amax|X| / 2688                         (1 when amax = 0)
 //     q      = amax_b / (6 * g)                       per 16 consecutive k

@@ -187,9 +187,10 @@ NVFP4_API nvfp4_status nvfp4_pack_scales(const uint8_t* s_plain, int rows, int K
 NVFP4_API size_t nvfp4_quantize_workspace_bytes(void);
 
 /* Two-level NVFP4 quantisation of a BF16 matrix, the encoding the W4A4 product
- * consumes (the FFN-down workload: "per-16 scale = amax/6 rounded to E4M3 and a
- * per-tensor FP32 scale = tensor amax/(6*448)", read as two levels: the block
- * scale relative to the per-tensor one).  Every step is an IEEE FP32 operation
+ * consumes (the FFN-down workload's: an E4M3 scale per 16 elements from their
+ * largest magnitude over 6, taken relative to an FP32 per-tensor scale from the
+ * tensor's largest magnitude over 6 x 448; metrale_circuit `hardware::exec`
+ * module doc, bullet 1, the NVFP4 row, for the format).  Every step is an IEEE FP32 operation
  * rounded to nearest even, in this order:
  *     g    = amax|X| / 2688                (g = 1 when X is all zero)
  *     s_b  = E4M3(amax_b / (6 g))          per 16 consecutive k of a row,

@@ -4,9 +4,10 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this module; the GPU library never does, and this file
 shares no code with it.
 
-What it computes (the FFN-down workload's quantisation, "per-16 scale = amax/6
-rounded to E4M3 and a per-tensor FP32 scale = tensor amax/(6*448)", in the
-two-level reading: the block scale is taken relative to the per-tensor scale).
+What it computes (the FFN-down workload's quantisation: each run of 16 elements
+gets an E4M3 scale from its largest magnitude over 6, and the tensor an FP32
+scale from its largest magnitude over 6 x 448; in the two-level reading the block
+scale is taken relative to the per-tensor scale).
 The pages fix FP32 for the per-tensor scale, so every step below is an IEEE
 FP32 operation, round to nearest even, in this order:
 
