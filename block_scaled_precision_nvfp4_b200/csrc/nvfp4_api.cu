@@ -105,9 +105,9 @@ bool class_compiles_fp8_exact_kernel(int arch) { return arch == 100; }
 bool class_compiles_bf16_widen_kernel(int arch) { return arch == 100; }
 
 // fp4_fallback: an NVFP4 activation on a class without an FP4 block-scale
-// kernel.  NoFp4Kernel where the class has the FP4 MMA and only the kernel is
-// missing; else the exact FP8 path where the class has the FP8 MMA (and this
-// library's exact-path kernel); else no path.
+// kernel.  NoFp4Kernel where the class's tensor cores do FP4 but this library
+// compiles no kernel for it; else the exact FP8 path where the class has the FP8
+// MMA (and this library's exact-path kernel); else no path.
 nvfp4_exec fp4_fallback(int arch) {
     if (class_has_fp4_mma(arch)) return NVFP4_EXEC_NO_FP4_KERNEL;
     if (class_has_fp8_mma(arch) && class_compiles_fp8_exact_kernel(arch)) return NVFP4_EXEC_FP8_EXACT;

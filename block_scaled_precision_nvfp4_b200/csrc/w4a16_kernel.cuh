@@ -1,8 +1,9 @@
 // w4a16_kernel.cuh -- BF16 activations x NVFP4 weights widened in registers.
 //
-// The "BF16 activations: BF16 MMA, any weight format widened in registers"
-// row of the metrale_circuit `hardware::exec` module doc, bullet 1, for the
-// decode shape (a handful of tokens, HBM-bound on the weight stream).
+// The BF16 row of the metrale_circuit `hardware::exec` module doc, bullet 1
+// (BF16 activations on the BF16 MMA, the weights widened to BF16 in registers
+// whatever their format), for the decode shape (a handful of tokens, HBM-bound
+// on the weight stream).
 //
 // Design (one wave of CTAs, one per SM, no cluster, no workspace):
 //  * the weight rows are cut into blocks of 8 (the MMA's N); CTA c takes a
