@@ -9,9 +9,10 @@
  * where a, w are E2M1 (FP4) values, g runs over groups of 16 consecutive k,
  * sA, sW are E4M3 group scales, alpha = gA*gW is the product of the two FP32
  * per-tensor scales, accumulation is FP32 and the output is BF16 (round to
- * nearest even).  The declared formats are never widened ("no silent upcast",
- * module doc, Invariants): a pair with no native or exact path is reported as
- * NVFP4_EXEC_NO_PATH and every matmul entry point refuses it.
+ * nearest even).  The declared formats are never widened (module doc,
+ * Invariants): a format pair that has neither a native kernel nor an exact
+ * conversion here is reported as NVFP4_EXEC_NO_PATH, and every matmul entry
+ * point refuses it.
  *
  * Layouts (all row-major, contiguous, no padding):
  *   A      uint8 [M][K/2]   E2M1 codes, two per byte, even k in the low nibble
@@ -112,8 +113,8 @@ NVFP4_API nvfp4_exec nvfp4_exec_of(int device, nvfp4_fmt weight, nvfp4_fmt activ
 
 /* fp4_fallback (metrale_circuit `hardware::exec`, fp4_fallback): how an NVFP4
  * activation runs on class `sm_arch` when no FP4 block-scale kernel is
- * compiled for it.  NO_FP4_KERNEL where the class has the FP4 MMA and only the
- * kernel is missing (sm_100 with the switch below, sm_101/103/110/120/121);
+ * compiled for it.  NO_FP4_KERNEL where the class's tensor cores do FP4 but no
+ * kernel for it is compiled (sm_100 with the switch below, sm_101/103/110/120/121);
  * FP8_EXACT on a class without the FP4 MMA that has the FP8 MMA and this
  * library's exact-path kernel (none besides sm_100, so in practice never);
  * NO_PATH otherwise.  Pure function; usable without a GPU. */
