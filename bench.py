@@ -54,7 +54,34 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true", help="time the eager launches only")
+    p.add_argument("--no-other-paths", action="store_true",
+                   help="on one GPU, the default FFN-down line also times the other paths "
+                        "(short runs, summarised under other_paths); this skips them")
     return p.parse_args()
+
+
+# the paths the default one-GPU line also times, each in its own short run
+OTHER_PATHS = ["grouped", "moe", "w4a8", "via_fp8", "w4a16", "quantize"]
+
+
+def other_paths(args):
+    """{workload: summary} of a short run of each other path (errors recorded, not raised)."""
+    out = {}
+    for w in OTHER_PATHS:
+        sub = argparse.Namespace(**vars(args))
+        sub.workload, sub.steps, sub.warmup = w, max(1, min(args.steps, 30)), 3
+        sub.no_e2e = sub.no_cpu_baseline = sub.no_other_paths = True
+        try:
+            d = run_ours(sub, emit=False)
+            r = d.get("roofline", {})
+            out[w] = {"metric": d["metric"], "value": d["value"], "unit": d["unit"],
+                      "ms_per_step": d["ms_per_step"], "steps": d["steps"],
+                      "roofline": {k: r.get(k) for k in ("bound", "achieved", "peak", "unit", "frac",
+                                                         "traffic", "kernel", "kernel_ms")},
+                      "gpu_launches": d.get("gpu_launches"), "clocks": d.get("clocks")}
+        except Exception as exc:  # keep the headline line; report what failed
+            out[w] = {"error": f"{type(exc).__name__}: {str(exc)[:200]}"}
+    return out
 
 
 def peaks():
@@ -412,7 +439,7 @@ def profiled_traffic(workload_name, path):
     return None
 
 
-def run_ours(args):
+def run_ours(args, emit=True):
     import torch
     import torch.distributed as dist
     import block_scaled_precision_nvfp4_b200 as nv
@@ -850,20 +877,24 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl_)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
     graph = None  # release the captured step before the process group goes
+    if (emit and world == 1 and args.workload == "ffn_down"
+            and not getattr(args, "no_other_paths", False)):
+        line["other_paths"] = other_paths(args)
+    if rank == 0 and emit:
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-    return 0
+    return line
 
 
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
-    return run_ours(args)
+    run_ours(args)
+    return 0
 
 
 if __name__ == "__main__":
