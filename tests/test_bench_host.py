@@ -93,3 +93,31 @@ def test_reference_arm_prints_its_line_on_the_host():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"].startswith("ffn_down")
+
+
+def test_other_paths_summarise_each_run_and_record_failures(monkeypatch):
+    """The default line's other_paths: one short run per other workload (at most 30
+    timed steps, 3 warm-up, no e2e or CPU baseline), summarised; a failing path is
+    recorded with its error instead of stopping the line."""
+    b = _bench()
+    seen = []
+
+    def fake_run(sub, emit=True):
+        assert emit is False
+        seen.append((sub.workload, sub.steps, sub.warmup, sub.no_e2e, sub.no_cpu_baseline,
+                     sub.no_other_paths))
+        if sub.workload == "w4a8":
+            raise RuntimeError("boom")
+        return {"metric": "m", "value": 1.0, "unit": "u", "ms_per_step": 0.5, "steps": sub.steps,
+                "roofline": {"frac": 0.5, "bound": "tensor"}, "gpu_launches": 2, "clocks": {}}
+
+    monkeypatch.setattr(b, "run_ours", fake_run)
+    args = types.SimpleNamespace(workload="ffn_down", steps=200, warmup=10, no_e2e=False,
+                                 no_cpu_baseline=False, no_other_paths=False, gpus=1,
+                                 impl="ours", no_graph=False)
+    out = b.other_paths(args)
+    assert [s[0] for s in seen] == b.OTHER_PATHS
+    assert all(s[1:] == (30, 3, True, True, True) for s in seen)
+    assert out["w4a8"] == {"error": "RuntimeError: boom"}
+    assert out["grouped"]["value"] == 1.0 and out["grouped"]["roofline"]["frac"] == 0.5
+    assert args.steps == 200 and args.no_e2e is False  # the headline's own arguments untouched
